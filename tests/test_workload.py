@@ -1,0 +1,50 @@
+"""The seeded input generator: shapes, dtypes, determinism, draw order, RoPE."""
+import torch
+
+import workload
+
+
+def test_shapes_and_dtypes():
+    w = workload.CONFIGS["tiny_fp32_n256"]
+    x = workload.generate(w)
+    assert list(x) == ["q"]
+    assert x["q"][0].shape == (1, 1, 256, 64) and x["q"][0].dtype == torch.float32
+    g = workload.Workload("g", B=2, H=4, H_kv=2, N=16, d=8, dtype="bf16", causal=True,
+                          relations=("q", "k", "v"), rope_base=5e5, pi_factor=4.0, v_noise=0.05,
+                          seed=4)
+    x = workload.generate(g)
+    assert x["q"][1].shape == (2, 4, 16, 8) and x["k"][0].shape == (2, 2, 16, 8)
+    assert x["v"][1].dtype == torch.bfloat16 and x["v"][1].is_contiguous()
+    assert g.n_units == 2 * (4 + 2 + 2) and len(workload.unit_list(g)) == g.n_units
+
+
+def test_deterministic_and_subset_independent():
+    g = workload.Workload("g", B=1, H=2, H_kv=2, N=32, d=16, dtype="bf16", causal=True,
+                          relations=("q", "k", "v"), rope_base=1e4, pi_factor=8.0, v_noise=0.1,
+                          seed=7)
+    a, b = workload.generate(g), workload.generate(g)
+    for r in "qkv":
+        assert torch.equal(a[r][0], b[r][0]) and torch.equal(a[r][1], b[r][1])
+    only_v = workload.generate(workload.Workload(**{**g.__dict__, "relations": ("v",)}))
+    assert torch.equal(only_v["v"][1], a["v"][1])
+
+
+def test_rope_and_pi():
+    g = workload.tiny_custom(N=64, d=8, dtype="fp32", seed=3, pi_factor=4.0)
+    xt, xs = workload.generate(g)["q"]
+    # position 0 is not rotated: teacher and student agree there
+    assert torch.equal(xt[..., 0, :], xs[..., 0, :])
+    assert not torch.equal(xt[..., 5, :], xs[..., 5, :])
+    # rotation preserves norms (up to the final rounding to fp32)
+    torch.testing.assert_close(xt.norm(dim=-1), xs.norm(dim=-1), rtol=1e-6, atol=1e-6)
+    # student at p/4 equals a teacher-style rotation at p/4
+    u = torch.randn(1, 1, 64, 8, generator=torch.Generator().manual_seed(3))
+    ref = workload.rope_rotate(u, torch.arange(64, dtype=torch.float64) / 4.0, 1e4).float()
+    torch.testing.assert_close(xs, ref, rtol=0, atol=0)
+
+
+def test_v_noise_level():
+    w = workload.Workload("v", B=1, H=2, H_kv=2, N=512, d=64, dtype="fp32", causal=True,
+                          relations=("v",), rope_base=1e4, pi_factor=8.0, v_noise=0.1, seed=2)
+    vt, vs = workload.generate(w)["v"]
+    assert abs(float((vs - vt).std()) - 0.1) < 0.005

@@ -1,0 +1,6 @@
+"""Seeded synthetic inputs shared by the oracle tests, the GPU tests and the bench."""
+from .synthetic import (CONFIGS, SWEEP_N, Workload, gaussian_pair, generate, get_config,
+                        rope_rotate, sweep_config, tiny_custom, unit_list)
+
+__all__ = ["CONFIGS", "SWEEP_N", "Workload", "gaussian_pair", "generate", "get_config",
+           "rope_rotate", "sweep_config", "tiny_custom", "unit_list"]
