@@ -1,0 +1,403 @@
+// Host side of the C ABI declared in include/relkl.h: argument validation,
+// TMA descriptor encoding, kernel selection and launch.  No allocation and no
+// state survives a call except two process-wide settings (the wait timeout
+// and a per-device SM-count cache).
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/relkl.h"
+#include "relkl_device.cuh"
+#include "relkl_params.h"
+
+namespace relkl {
+cudaError_t tc_launch_fwd(const TcParams& p, int d, int grid, cudaStream_t stream);
+cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t stream);
+cudaError_t simt_launch_fwd(const SimtParams& p, cudaStream_t stream);
+cudaError_t simt_launch_bwd(const SimtParams& p, cudaStream_t stream);
+cudaError_t launch_zero(float* ptr, int64_t n, int num_sms, cudaStream_t stream);
+}  // namespace relkl
+
+using namespace relkl;
+
+namespace {
+
+constexpr size_t kWorkspaceBytes = 256;
+std::atomic<unsigned long long> g_timeout_ns{2000000000ull};
+thread_local int32_t g_last_cuda = 0;
+
+relkl_status cuda_fail(cudaError_t e) {
+  g_last_cuda = static_cast<int32_t>(e);
+  return RELKL_ERR_CUDA;
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime so the
+// library needs no link-time dependency on libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+EncodeTiledFn encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+struct DevInfo {
+  int sms = 0;
+  int major = 0;
+};
+DevInfo g_dev[64];
+std::mutex g_dev_mu;
+
+relkl_status device_info(DevInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return RELKL_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_dev[dev].sms == 0) {
+    int sms = 0, major = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) !=
+        cudaSuccess)
+      return cuda_fail(e);
+    g_dev[dev].sms = sms;
+    g_dev[dev].major = major;
+  }
+  *out = g_dev[dev];
+  return RELKL_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t n_units(const relkl_desc& d) { return static_cast<int64_t>(d.B) * d.H; }
+
+relkl_status check_desc(const relkl_desc* d) {
+  if (!d) return RELKL_ERR_INVALID;
+  if (d->B < 0 || d->H < 0 || d->N < 0 || d->d < 1) return RELKL_ERR_INVALID;
+  if (d->dtype != RELKL_BF16 && d->dtype != RELKL_FP32) return RELKL_ERR_INVALID;
+  if (d->causal != 0 && d->causal != 1) return RELKL_ERR_INVALID;
+  if (d->reserved != 0) return RELKL_ERR_INVALID;
+  if (!(d->scale >= 0.f) || !std::isfinite(d->scale)) return RELKL_ERR_INVALID;
+  if (d->stride[3] != 1) return RELKL_ERR_INVALID;
+  for (int i = 0; i < 3; ++i)
+    if (d->stride[i] < 0) return RELKL_ERR_INVALID;
+  if (d->d > 128) return RELKL_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->N) * d->d >= (int64_t(1) << 31)) return RELKL_ERR_UNSUPPORTED;
+  if (n_units(*d) * d->N >= (int64_t(1) << 40)) return RELKL_ERR_UNSUPPORTED;
+  return RELKL_OK;
+}
+
+bool tc_shape(const relkl_desc& d) {
+  return d.dtype == RELKL_BF16 && (d.d == 64 || d.d == 128);
+}
+
+// Tensor-core path needs 16-byte aligned bases and strides (TMA).
+bool tc_layout_ok(const relkl_desc& d, const void* xt, const void* xs) {
+  if (!aligned(xt, 16) || !aligned(xs, 16)) return false;
+  for (int i = 0; i < 3; ++i)
+    if ((d.stride[i] * 2) % 16 != 0) return false;
+  return true;
+}
+
+float logit_scale(const relkl_desc& d) {
+  return d.scale > 0.f ? d.scale : 1.0f / std::sqrt(static_cast<float>(d.d));
+}
+
+relkl_status encode_x(CUtensorMap* m, const relkl_desc& d, const void* x) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return RELKL_ERR_CUDA;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.d), static_cast<cuuint64_t>(d.N),
+                              static_cast<cuuint64_t>(d.H), static_cast<cuuint64_t>(d.B)};
+  // a dimension of extent 1 may carry any stride; give it a legal one
+  auto stride_or = [&](int i, int64_t fallback) {
+    return static_cast<cuuint64_t>((d.stride[i] > 0 ? d.stride[i] : fallback) * 2);
+  };
+  const int64_t row = d.stride[2] > 0 ? d.stride[2] : d.d;
+  const cuuint64_t strides[3] = {stride_or(2, d.d), stride_or(1, row * d.N),
+                                 stride_or(0, row * d.N * d.H)};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RELKL_OK : RELKL_ERR_UNSUPPORTED;
+}
+
+relkl_status check_ws(const void* ws, size_t ws_bytes) {
+  if (!ws || ws_bytes < kWorkspaceBytes || !aligned(ws, 256)) return RELKL_ERR_WORKSPACE;
+  return RELKL_OK;
+}
+
+// Common validation of a multi-relation call.  Sets *empty when there is no
+// work at all.
+relkl_status check_multi(int32_t n_rel, const relkl_desc* descs, const void* const* xt,
+                         const void* const* xs, bool* empty) {
+  if (n_rel < 1 || n_rel > kMaxSeg || !descs || !xt || !xs) return RELKL_ERR_INVALID;
+  int64_t units = 0;
+  for (int r = 0; r < n_rel; ++r) {
+    relkl_status s = check_desc(&descs[r]);
+    if (s != RELKL_OK) return s;
+    const relkl_desc& a = descs[0];
+    const relkl_desc& b = descs[r];
+    if (a.N != b.N || a.d != b.d || a.dtype != b.dtype || a.causal != b.causal ||
+        a.scale != b.scale)
+      return RELKL_ERR_INVALID;
+    units += n_units(b);
+  }
+  if (units >= (int64_t(1) << 30)) return RELKL_ERR_UNSUPPORTED;
+  *empty = (units == 0 || descs[0].N == 0);
+  if (*empty) return RELKL_OK;
+  for (int r = 0; r < n_rel; ++r) {
+    if (n_units(descs[r]) == 0) continue;
+    if (!xt[r] || !xs[r]) return RELKL_ERR_INVALID;
+    const size_t es = descs[r].dtype == RELKL_BF16 ? 2 : 4;
+    if (!aligned(xt[r], es) || !aligned(xs[r], es)) return RELKL_ERR_INVALID;
+  }
+  return RELKL_OK;
+}
+
+bool use_tc(int32_t n_rel, const relkl_desc* descs, const void* const* xt, const void* const* xs) {
+  if (!tc_shape(descs[0])) return false;
+  for (int r = 0; r < n_rel; ++r)
+    if (n_units(descs[r]) && !tc_layout_ok(descs[r], xt[r], xs[r])) return false;
+  return true;
+}
+
+relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const* xt,
+                      const void* const* xs, TcParams* p, void* ws) {
+  std::memset(p, 0, sizeof(*p));
+  const relkl_desc& d0 = descs[0];
+  int seg = 0, ub = 0;
+  for (int r = 0; r < n_rel; ++r) {
+    if (n_units(descs[r]) == 0) continue;
+    TcSeg& s = p->seg[seg];
+    relkl_status st = encode_x(&s.tm_t, descs[r], xt[r]);
+    if (st != RELKL_OK) return st;
+    if ((st = encode_x(&s.tm_s, descs[r], xs[r])) != RELKL_OK) return st;
+    s.B = descs[r].B;
+    s.H = descs[r].H;
+    s.unit_begin = ub;
+    ub += static_cast<int>(n_units(descs[r]));
+    ++seg;
+  }
+  p->n_seg = seg;
+  p->N = d0.N;
+  p->nblk = (d0.N + 127) / 128;
+  p->n_pairs = (p->nblk + 1) / 2;
+  p->n_items = ub * p->n_pairs;
+  p->causal = d0.causal;
+  p->scale = logit_scale(d0);
+  p->sl2 = p->scale * 1.4426950408889634f;
+  p->status = reinterpret_cast<DevStatus*>(ws);
+  p->timeout_ns = g_timeout_ns.load();
+  return RELKL_OK;
+}
+
+relkl_status build_simt(int32_t n_rel, const relkl_desc* descs, const void* const* xt,
+                        const void* const* xs, SimtParams* p) {
+  std::memset(p, 0, sizeof(*p));
+  const relkl_desc& d0 = descs[0];
+  int seg = 0, ub = 0;
+  for (int r = 0; r < n_rel; ++r) {
+    if (n_units(descs[r]) == 0) continue;
+    SimtSeg& s = p->seg[seg];
+    s.xt = xt[r];
+    s.xs = xs[r];
+    s.sb = descs[r].stride[0];
+    s.sh = descs[r].stride[1];
+    s.sn = descs[r].stride[2];
+    s.B = descs[r].B;
+    s.H = descs[r].H;
+    s.unit_begin = ub;
+    ub += static_cast<int>(n_units(descs[r]));
+    ++seg;
+  }
+  p->n_seg = seg;
+  p->N = d0.N;
+  p->d = d0.d;
+  p->causal = d0.causal;
+  p->is_bf16 = d0.dtype == RELKL_BF16;
+  p->scale = logit_scale(d0);
+  p->n_units = ub;
+  return RELKL_OK;
+}
+
+// Index of relation r's segment (relations without units have none).
+template <class P>
+void set_seg_outputs(P* p, int32_t n_rel, const relkl_desc* descs, float* const* kl,
+                     float* const* stats, const float* const* stats_in, const float* const* dkl,
+                     float* const* dx) {
+  int seg = 0;
+  for (int r = 0; r < n_rel; ++r) {
+    if (n_units(descs[r]) == 0) continue;
+    auto& s = p->seg[seg++];
+    if (kl) s.kl = kl[r];
+    if (stats) s.stats = stats[r];
+    if (stats_in) s.stats = const_cast<float*>(stats_in[r]);
+    s.dkl = dkl ? dkl[r] : nullptr;
+    if (dx) s.dx = dx[r];
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t relkl_workspace_bytes(void) { return kWorkspaceBytes; }
+
+relkl_status relkl_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  relkl_status s = check_ws(ws, ws_bytes);
+  if (s != RELKL_OK) return s;
+  cudaError_t e = cudaMemsetAsync(ws, 0, kWorkspaceBytes, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
+}
+
+int32_t relkl_path_for(const relkl_desc* desc) {
+  if (check_desc(desc) != RELKL_OK) return 0;
+  return tc_shape(*desc) ? 1 : 2;
+}
+
+relkl_status relkl_fwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
+                           const void* const* x_s, float* const* kl, float* const* stats,
+                           void* ws, size_t ws_bytes, void* stream) {
+  bool empty = false;
+  relkl_status s = check_multi(n_rel, descs, x_t, x_s, &empty);
+  if (s != RELKL_OK || empty) return s;
+  if (!kl || !stats) return RELKL_ERR_INVALID;
+  for (int r = 0; r < n_rel; ++r)
+    if (n_units(descs[r]) && (!kl[r] || !stats[r] || !aligned(kl[r], 4) || !aligned(stats[r], 16)))
+      return RELKL_ERR_INVALID;
+  if ((s = check_ws(ws, ws_bytes)) != RELKL_OK) return s;
+  DevInfo dev;
+  if ((s = device_info(&dev)) != RELKL_OK) return s;
+  if (dev.major != 10) return RELKL_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (use_tc(n_rel, descs, x_t, x_s)) {
+    TcParams p;
+    if ((s = build_tc(n_rel, descs, x_t, x_s, &p, ws)) != RELKL_OK) return s;
+    set_seg_outputs(&p, n_rel, descs, kl, stats, nullptr, nullptr, nullptr);
+    const int grid = p.n_items < dev.sms ? p.n_items : dev.sms;
+    e = tc_launch_fwd(p, descs[0].d, grid, st);
+  } else {
+    SimtParams p;
+    build_simt(n_rel, descs, x_t, x_s, &p);
+    set_seg_outputs(&p, n_rel, descs, kl, stats, nullptr, nullptr, nullptr);
+    e = simt_launch_fwd(p, st);
+  }
+  return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
+}
+
+relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
+                           const void* const* x_s, const float* const* stats,
+                           const float* const* dkl, float* const* dx_s, void* ws,
+                           size_t ws_bytes, void* stream) {
+  bool empty = false;
+  relkl_status s = check_multi(n_rel, descs, x_t, x_s, &empty);
+  if (s != RELKL_OK || empty) return s;
+  if (!stats || !dx_s) return RELKL_ERR_INVALID;
+  for (int r = 0; r < n_rel; ++r) {
+    if (!n_units(descs[r])) continue;
+    if (!stats[r] || !dx_s[r] || !aligned(stats[r], 16) || !aligned(dx_s[r], 16))
+      return RELKL_ERR_INVALID;
+    if (dkl && dkl[r] && !aligned(dkl[r], 4)) return RELKL_ERR_INVALID;
+  }
+  if ((s = check_ws(ws, ws_bytes)) != RELKL_OK) return s;
+  DevInfo dev;
+  if ((s = device_info(&dev)) != RELKL_OK) return s;
+  if (dev.major != 10) return RELKL_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  const bool tc = use_tc(n_rel, descs, x_t, x_s);
+  TcParams tp;
+  SimtParams sp;
+  if (tc) {
+    if ((s = build_tc(n_rel, descs, x_t, x_s, &tp, ws)) != RELKL_OK) return s;
+    set_seg_outputs(&tp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);
+  } else {
+    build_simt(n_rel, descs, x_t, x_s, &sp);
+    set_seg_outputs(&sp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);
+  }
+  // dX_s is accumulated with atomics: clear it first (same stream)
+  for (int r = 0; r < n_rel; ++r) {
+    if (!n_units(descs[r])) continue;
+    const int64_t n = n_units(descs[r]) * descs[r].N * descs[r].d;
+    if ((e = launch_zero(dx_s[r], n, dev.sms, st)) != cudaSuccess) return cuda_fail(e);
+  }
+  if (tc) {
+    const int grid = tp.n_items < dev.sms ? tp.n_items : dev.sms;
+    e = tc_launch_bwd(tp, descs[0].d, grid, st);
+  } else {
+    e = simt_launch_bwd(sp, st);
+  }
+  return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
+}
+
+relkl_status relkl_fwd(const relkl_desc* desc, const void* x_t, const void* x_s, float* kl,
+                       float* stats, void* ws, size_t ws_bytes, void* stream) {
+  const void* xt[1] = {x_t};
+  const void* xs[1] = {x_s};
+  float* k[1] = {kl};
+  float* st[1] = {stats};
+  return relkl_fwd_qkv(1, desc, xt, xs, k, st, ws, ws_bytes, stream);
+}
+
+relkl_status relkl_bwd(const relkl_desc* desc, const void* x_t, const void* x_s,
+                       const float* stats, const float* dkl, float* dx_s, void* ws,
+                       size_t ws_bytes, void* stream) {
+  const void* xt[1] = {x_t};
+  const void* xs[1] = {x_s};
+  const float* st[1] = {stats};
+  const float* g[1] = {dkl};
+  float* dx[1] = {dx_s};
+  return relkl_bwd_qkv(1, desc, xt, xs, st, g, dx, ws, ws_bytes, stream);
+}
+
+relkl_status relkl_get_device_error(const void* ws, void* stream, uint32_t* where) {
+  if (where) *where = 0;
+  relkl_status s = check_ws(ws, kWorkspaceBytes);
+  if (s != RELKL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  DevStatus rec;
+  e = cudaMemcpy(&rec, ws, sizeof(rec), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (where) *where = rec.where;
+  return rec.code == 0 ? RELKL_OK : RELKL_ERR_TIMEOUT;
+}
+
+uint64_t relkl_set_wait_timeout_ns(uint64_t ns) { return g_timeout_ns.exchange(ns); }
+
+const char* relkl_status_string(relkl_status s) {
+  switch (s) {
+    case RELKL_OK: return "RELKL_OK";
+    case RELKL_ERR_INVALID: return "RELKL_ERR_INVALID: invalid argument";
+    case RELKL_ERR_UNSUPPORTED: return "RELKL_ERR_UNSUPPORTED: unsupported shape, layout or device";
+    case RELKL_ERR_CUDA: return "RELKL_ERR_CUDA: a CUDA call failed";
+    case RELKL_ERR_WORKSPACE: return "RELKL_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case RELKL_ERR_TIMEOUT: return "RELKL_ERR_TIMEOUT: a bounded device wait ran out";
+  }
+  return "RELKL_ERR_UNKNOWN";
+}
+
+int32_t relkl_last_cuda_error(void) { return g_last_cuda; }
+
+}  // extern "C"

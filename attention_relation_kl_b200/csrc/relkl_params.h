@@ -1,0 +1,65 @@
+// Kernel parameter blocks shared by the launch code and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+namespace relkl {
+
+struct DevStatus;
+
+constexpr int kMaxSeg = 3;   // relations per launch (Q, K, V)
+
+// One relation inside a launch.  Units of relation r are numbered
+// unit_begin .. unit_begin + B*H - 1, batch-major then head.
+struct TcSeg {
+  CUtensorMap tm_t;          // teacher [B,H,N,d] bf16, box 64 cols x 128 rows, 128B swizzle
+  CUtensorMap tm_s;          // student, same geometry
+  float* kl;                 // [B,H,N]
+  float* stats;              // [B,H,N,4]
+  const float* dkl;          // [B,H,N] or null (1/N)
+  float* dx;                 // [B,H,N,d] float32
+  int B, H;
+  int unit_begin;
+  int pad_;
+};
+
+struct TcParams {
+  TcSeg seg[kMaxSeg];
+  int n_seg;
+  int N;
+  int nblk;       // ceil(N / 128)
+  int n_pairs;    // ceil(nblk / 2): row blocks p and nblk-1-p form one work item
+  int n_items;    // units * n_pairs
+  int causal;
+  float scale;    // logit scale
+  float sl2;      // scale * log2(e)
+  DevStatus* status;
+  unsigned long long timeout_ns;
+};
+
+// CUDA-core float32 path: plain pointers with element strides.
+struct SimtSeg {
+  const void* xt;
+  const void* xs;
+  int64_t sb, sh, sn;        // element strides of B, H, N (d is contiguous)
+  float* kl;
+  float* stats;
+  const float* dkl;
+  float* dx;
+  int B, H;
+  int unit_begin;
+  int pad_;
+};
+
+struct SimtParams {
+  SimtSeg seg[kMaxSeg];
+  int n_seg;
+  int N, d;
+  int causal;
+  int is_bf16;
+  float scale;
+  int n_units;
+};
+
+}  // namespace relkl

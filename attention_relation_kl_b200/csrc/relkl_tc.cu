@@ -1,0 +1,809 @@
+// tcgen05 / TMA kernels (sm_100a) for the linear-memory relation KL.
+//
+// LinearARD (arXiv 2604.00004; pith.science verdict, pith_extraction.
+// key_machinery) computes, per (batch, head, relation) unit,
+//   Z_m = X_m X_m^T * s + M,  R_m = softmax_rows(Z_m),  kl_i = KL(R_t(i,:) || R_s(i,:)),
+// keeping only O(N) row statistics (Phase 1) and recomputing the logit tiles
+// in the backward pass (Phase 2), where G = dkl (R_s - R_t) and
+// dX_s = s (G + G^T) X_s.
+//
+// Both kernels are persistent (one CTA per SM, static schedule) and
+// warp-specialised:
+//   * one TMA warp streams 128-row bf16 tiles of X_t and X_s into 128-byte
+//     swizzled shared memory (the row block I stays resident, column blocks J
+//     pass through a two-stage ring);
+//   * one MMA warp issues tcgen05.mma (kind::f16, M=128) whose fp32
+//     accumulators live in tensor memory: the teacher and student logit tiles
+//     side by side, and in the backward also dX_I += G X_s[J] and
+//     P = G^T X_s[I];
+//   * two "row" warpgroups read the logit tiles from TMEM (one column half
+//     each) and do the per-entry work: the shared-max online softmax and KL
+//     sums in the forward, the gradient tile G (bf16, written to shared
+//     memory as an MMA operand) in the backward;
+//   * in the backward an epilogue warpgroup adds P into dX[J] and, at the end
+//     of a row block, the dX_I accumulator into dX[I] with float32 atomics.
+//
+// Work items pair row block p with row block nblk-1-p of the same unit, so
+// every causal item holds nblk+1 column tiles and the static round-robin over
+// items is balanced; consecutive items belong to the same unit, which keeps
+// the unit's X tiles and dX rows resident in L2 while its items run.
+//
+// Every mbarrier wait is bounded (see relkl_device.cuh): a wait that runs out
+// records its site in the caller's workspace, and every role then leaves its
+// loop, waits for its own copies and MMAs in flight and the CTA frees its TMEM
+// and exits.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "relkl_device.cuh"
+#include "relkl_params.h"
+
+namespace relkl {
+
+constexpr int BM = 128;        // rows of a row block (TMEM lanes)
+constexpr int BN = 128;        // columns of a logit tile
+constexpr int BOX = 128 * 128;  // bytes of one 128-row x 64-col bf16 box
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr unsigned long long kDrainNs = 200000000ull;  // 0.2 s for in-flight copies
+
+struct Unit {
+  const TcSeg* seg;
+  int b, h;
+  long long row0;  // (b*H + h) * N : first row of the unit in [B,H,N] arrays
+};
+
+__device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
+  int r = 0;
+#pragma unroll
+  for (int k = 1; k < kMaxSeg; ++k)
+    if (k < p.n_seg && u >= p.seg[k].unit_begin) r = k;
+  const TcSeg* s = &p.seg[r];
+  const int local = u - s->unit_begin;
+  Unit out;
+  out.seg = s;
+  out.b = local / s->H;
+  out.h = local - out.b * s->H;
+  out.row0 = (static_cast<long long>(out.b) * s->H + out.h) * p.N;
+  return out;
+}
+
+// Row blocks of one work item: pass 0 is the longer block nblk-1-p, pass 1
+// (absent when both coincide) is block p.
+__device__ __forceinline__ int item_passes(const TcParams& p, int pp) {
+  return (pp == p.nblk - 1 - pp) ? 1 : 2;
+}
+__device__ __forceinline__ int pass_block(const TcParams& p, int pp, int pass) {
+  return pass == 0 ? p.nblk - 1 - pp : pp;
+}
+__device__ __forceinline__ int n_col_tiles(const TcParams& p, int I) {
+  return p.causal ? I + 1 : p.nblk;
+}
+
+// Issue the K-loop of one M=128 x N=128 logit tile: acc = A_tile * B_tile^T
+// with both operands K-major (rows of X, d contiguous), K = D.
+template <int D>
+__device__ __forceinline__ void issue_logits(uint32_t acc, uint32_t a_base, uint32_t b_base) {
+  constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint32_t off = (k >> 2) * BOX + (k & 3) * 32;
+    umma_bf16(acc, sw128_desc(a_base + off, 16, 1024), sw128_desc(b_base + off, 16, 1024), idesc,
+              k > 0 ? 1u : 0u);
+  }
+}
+
+// =========================================================================
+//                                FORWARD
+// =========================================================================
+template <int D>
+struct FwdSmem {
+  static constexpr int TILE = BM * D * 2;
+  static constexpr int XT_I = 0;
+  static constexpr int XS_I = TILE;
+  static constexpr int RING = 2 * TILE;              // stage k: xt at RING + 2k*TILE, xs after it
+  static constexpr int STAGES = 2;
+  static constexpr int MERGE = RING + STAGES * 2 * TILE;  // float4 per row
+  static constexpr int BARS = MERGE + BM * 16;
+  // barriers: full_I, empty_I, full_J[2], empty_J[2], tf[2], te[2], mfull, mempty, drain
+  static constexpr int NBAR = 13;
+  static constexpr int MISC = BARS + NBAR * 8;       // tmem base (u32) + abort flag (int)
+  static constexpr int BYTES = MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;         // slack for 1024-byte alignment
+};
+
+constexpr int FWD_THREADS = 320;   // warps 0-7 rows, 8 TMA, 9 MMA
+
+template <int D>
+__global__ void __launch_bounds__(FWD_THREADS, 1)
+relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
+  using L = FwdSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t bar0 = base + L::BARS;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1);
+  auto FULL_J = [&](int s) { return BAR(2 + s); };
+  auto EMPTY_J = [&](int s) { return BAR(4 + s); };
+  auto TF = [&](int b) { return BAR(6 + b); };
+  auto TE = [&](int b) { return BAR(8 + b); };
+  const uint32_t MFULL = BAR(10), MEMPTY = BAR(11), DRAIN = BAR(12);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
+  float4* merge = reinterpret_cast<float4*>(gbase + L::MERGE);
+
+  WaitCtl wc{p.status, abort_flag, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(FULL_I, 1);
+    mbar_init(EMPTY_I, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(FULL_J(s), 1);
+      mbar_init(EMPTY_J(s), 1);
+      mbar_init(TF(s), 1);
+      mbar_init(TE(s), 8);
+    }
+    mbar_init(MFULL, 4);
+    mbar_init(MEMPTY, 4);
+    mbar_init(DRAIN, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      for (int s = 0; s < p.n_seg; ++s) {
+        tma_prefetch_desc(&p.seg[s].tm_t);
+        tma_prefetch_desc(&p.seg[s].tm_s);
+      }
+      uint32_t nI = 0, nJ = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        const Unit U = decode_unit(p, u);
+        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+          const int I = pass_block(p, pp, pass);
+          if (!(ok = mbar_wait(EMPTY_I, (nI & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
+          mbar_arrive_expect_tx(FULL_I, 2 * L::TILE);
+#pragma unroll
+          for (int b = 0; b < D / 64; ++b) {
+            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, I * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, I * BM, U.h, U.b);
+          }
+          ++nI;
+          const int nT = n_col_tiles(p, I);
+          for (int J = 0; J < nT; ++J) {
+            const int st = nJ & 1;
+            if (!(ok = mbar_wait(EMPTY_J(st), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
+            const uint32_t xt = base + L::RING + st * 2 * L::TILE;
+            mbar_arrive_expect_tx(FULL_J(st), 2 * L::TILE);
+#pragma unroll
+            for (int b = 0; b < D / 64; ++b) {
+              tma_load_4d(xt + b * BOX, &U.seg->tm_t, FULL_J(st), b * 64, J * BN, U.h, U.b);
+              tma_load_4d(xt + L::TILE + b * BOX, &U.seg->tm_s, FULL_J(st), b * 64, J * BN, U.h,
+                          U.b);
+            }
+            ++nJ;
+          }
+        }
+      }
+      // wait for the copies still in flight before the CTA may exit
+      if (nI) mbar_wait_drain(FULL_I, (nI - 1) & 1, kDrainNs);
+      for (int st = 0; st < 2; ++st) {
+        const uint32_t arms = (nJ + 1 - st) / 2;
+        if (arms) mbar_wait_drain(FULL_J(st), (arms - 1) & 1, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      uint32_t nI = 0, nJ = 0, nt = 0;
+      bool ok = true, issued = false;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        (void)u;
+        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+          const int I = pass_block(p, pp, pass);
+          if (!(ok = mbar_wait(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
+          const int nT = n_col_tiles(p, I);
+          for (int J = 0; J < nT; ++J) {
+            const int st = nJ & 1;
+            const int buf = nt & 1;
+            if (!(ok = mbar_wait(FULL_J(st), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+            if (!(ok = mbar_wait(TE(buf), ((nt >> 1) & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
+            tc_fence_after();
+            const uint32_t xt = base + L::RING + st * 2 * L::TILE;
+            const uint32_t acc = tmem + buf * 256;
+            issue_logits<D>(acc, base + L::XT_I, xt);
+            issue_logits<D>(acc + 128, base + L::XS_I, xt + L::TILE);
+            issued = true;
+            umma_commit(EMPTY_J(st));
+            umma_commit(TF(buf));
+            ++nJ;
+            ++nt;
+          }
+          if (!ok) break;
+          umma_commit(EMPTY_I);
+          ++nI;
+        }
+      }
+      if (issued) {
+        umma_commit(DRAIN);
+        mbar_wait_drain(DRAIN, 0, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------- row warpgroups
+    const int q = warp & 3;      // TMEM lane quarter
+    const int half = warp >> 2;  // column half of each tile
+    const int r = q * 32 + lane;
+    const float sl2 = p.sl2;
+    uint32_t nt = 0, nm = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      const Unit U = decode_unit(p, u);
+      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+        const int I = pass_block(p, pp, pass);
+        const int row = I * BM + r;
+        const int nT = n_col_tiles(p, I);
+        float m_run = -INFINITY;
+        float S[4] = {0.f, 0.f, 0.f, 0.f}, C[4] = {0.f, 0.f, 0.f, 0.f},
+              A[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int J = 0; J < nT; ++J) {
+          const int buf = nt & 1;
+          ok = mbar_wait(TF(buf), (nt >> 1) & 1, wc, W_SM_S_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + half * 64;
+          float t0[32], s0[32], t1[32], s1[32];
+          tmem_ld32(ta, t0);
+          tmem_ld32(ta + 128, s0);
+          tmem_ld32(ta + 32, t1);
+          tmem_ld32(ta + 160, s1);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(TE(buf));
+          ++nt;
+
+          const int col0 = J * BN + half * 64;
+          const bool need_mask = (p.causal && J == I) || (col0 + 64 > p.N);
+          if (!need_mask) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              mx = fmaxf(mx, fmaxf(fmaxf(t0[k], s0[k]), fmaxf(t1[k], s1[k])));
+            if (mx > m_run) {
+              const float a = ex2_approx((m_run - mx) * sl2);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                S[k] *= a;
+                C[k] *= a;
+                A[k] *= a;
+              }
+              m_run = mx;
+            }
+            const float nb = -m_run * sl2;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const float et = ex2_approx(fmaf(t0[k], sl2, nb));
+              const float es = ex2_approx(fmaf(s0[k], sl2, nb));
+              S[k & 3] += et;
+              C[k & 3] += es - et;
+              A[k & 3] = fmaf(et, t0[k] - s0[k], A[k & 3]);
+            }
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const float et = ex2_approx(fmaf(t1[k], sl2, nb));
+              const float es = ex2_approx(fmaf(s1[k], sl2, nb));
+              S[k & 3] += et;
+              C[k & 3] += es - et;
+              A[k & 3] = fmaf(et, t1[k] - s1[k], A[k & 3]);
+            }
+          } else {
+            // diagonal or ragged tile: per-entry predicate
+            const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;  // last allowed column
+            float mx = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              if (col0 + k <= lim) mx = fmaxf(mx, fmaxf(t0[k], s0[k]));
+              if (col0 + 32 + k <= lim) mx = fmaxf(mx, fmaxf(t1[k], s1[k]));
+            }
+            if (mx > m_run) {
+              const float a = ex2_approx((m_run - mx) * sl2);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                S[k] *= a;
+                C[k] *= a;
+                A[k] *= a;
+              }
+              m_run = mx;
+            }
+            if (m_run > -INFINITY) {
+              const float nb = -m_run * sl2;
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                if (col0 + k <= lim) {
+                  const float et = ex2_approx(fmaf(t0[k], sl2, nb));
+                  const float es = ex2_approx(fmaf(s0[k], sl2, nb));
+                  S[k & 3] += et;
+                  C[k & 3] += es - et;
+                  A[k & 3] = fmaf(et, t0[k] - s0[k], A[k & 3]);
+                }
+                if (col0 + 32 + k <= lim) {
+                  const float et = ex2_approx(fmaf(t1[k], sl2, nb));
+                  const float es = ex2_approx(fmaf(s1[k], sl2, nb));
+                  S[k & 3] += et;
+                  C[k & 3] += es - et;
+                  A[k & 3] = fmaf(et, t1[k] - s1[k], A[k & 3]);
+                }
+              }
+            }
+          }
+        }
+        if (!ok) break;
+        const float Sx = (S[0] + S[1]) + (S[2] + S[3]);
+        const float Cx = (C[0] + C[1]) + (C[2] + C[3]);
+        const float Ax = (A[0] + A[1]) + (A[2] + A[3]);
+        // merge the two column halves through shared memory
+        if (half == 1) {
+          ok = mbar_wait(MEMPTY, (nm & 1) ^ 1, wc, W_SM_S_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          merge[r] = make_float4(m_run, Sx, Cx, Ax);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(MFULL);
+        } else {
+          ok = mbar_wait(MFULL, nm & 1, wc, W_SM_S_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          const float4 o = merge[r];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(MEMPTY);
+          const float M = fmaxf(m_run, o.x);
+          const float a0 = ex2_approx((m_run - M) * sl2);
+          const float a1 = ex2_approx((o.x - M) * sl2);
+          const float St = Sx * a0 + o.y * a1;
+          const float Ct = Cx * a0 + o.z * a1;
+          const float At = Ax * a0 + o.w * a1;
+          if (row < p.N) {
+            const float mz = M * p.scale;
+            const float lse_t = mz + logf(St);
+            const float rc = Ct / St;
+            const float l1 = log1pf(rc);
+            const float w = p.scale * At / St;
+            const long long g = U.row0 + row;
+            U.seg->kl[g] = w + l1;
+            reinterpret_cast<float4*>(U.seg->stats)[g] = make_float4(mz, lse_t, lse_t + l1, w);
+          }
+        }
+        ++nm;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// =========================================================================
+//                                BACKWARD
+// =========================================================================
+template <int D>
+struct BwdSmem {
+  static constexpr int TILE = BM * D * 2;
+  static constexpr int XT_I = 0;
+  static constexpr int XS_I = TILE;
+  static constexpr int XT_R = 2 * TILE;            // teacher ring, 2 stages
+  static constexpr int XS_R = 4 * TILE;            // student ring, 2 stages
+  static constexpr int G = 6 * TILE;               // 128 x 128 bf16 gradient tile (two boxes)
+  static constexpr int BARS = G + 2 * BOX;
+  // full_I, empty_I, fullT[2], emptyT[2], fullS[2], emptyS[2], s_full, s_empty,
+  // g_full, g_empty, p_full, p_empty, dxi_full, dxi_empty, drain
+  static constexpr int NBAR = 19;
+  static constexpr int MISC = BARS + NBAR * 8;
+  static constexpr int BYTES = MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+};
+
+constexpr int BWD_THREADS = 448;   // warps 0-7 rows, 8-11 epilogue, 12 TMA, 13 MMA
+
+template <int D>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
+  using L = BwdSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t bar0 = base + L::BARS;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1);
+  auto FULL_T = [&](int s) { return BAR(2 + s); };
+  auto EMPTY_T = [&](int s) { return BAR(4 + s); };
+  auto FULL_S = [&](int s) { return BAR(6 + s); };
+  auto EMPTY_S = [&](int s) { return BAR(8 + s); };
+  const uint32_t S_FULL = BAR(10), S_EMPTY = BAR(11), G_FULL = BAR(12), G_EMPTY = BAR(13);
+  const uint32_t P_FULL = BAR(14), P_EMPTY = BAR(15), DXI_FULL = BAR(16), DXI_EMPTY = BAR(17);
+  const uint32_t DRAIN = BAR(18);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
+
+  WaitCtl wc{p.status, abort_flag, p.timeout_ns};
+
+  // TMEM columns
+  constexpr uint32_t T_ST = 0, T_SS = 128, T_DXI = 256, T_P = 256 + D;
+
+  if (threadIdx.x == 0) {
+    mbar_init(FULL_I, 1);
+    mbar_init(EMPTY_I, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(FULL_T(s), 1);
+      mbar_init(EMPTY_T(s), 1);
+      mbar_init(FULL_S(s), 1);
+      mbar_init(EMPTY_S(s), 1);
+    }
+    mbar_init(S_FULL, 1);
+    mbar_init(S_EMPTY, 8);
+    mbar_init(G_FULL, 8);
+    mbar_init(G_EMPTY, 1);
+    mbar_init(P_FULL, 1);
+    mbar_init(P_EMPTY, 4);
+    mbar_init(DXI_FULL, 1);
+    mbar_init(DXI_EMPTY, 4);
+    mbar_init(DRAIN, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 12) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      for (int s = 0; s < p.n_seg; ++s) {
+        tma_prefetch_desc(&p.seg[s].tm_t);
+        tma_prefetch_desc(&p.seg[s].tm_s);
+      }
+      uint32_t nI = 0, nJ = 0;
+      uint32_t armsT[2] = {0, 0}, armsS[2] = {0, 0};   // loads issued per ring stage
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        const Unit U = decode_unit(p, u);
+        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+          const int I = pass_block(p, pp, pass);
+          if (!(ok = mbar_wait(EMPTY_I, (nI & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
+          mbar_arrive_expect_tx(FULL_I, 2 * L::TILE);
+#pragma unroll
+          for (int b = 0; b < D / 64; ++b) {
+            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, I * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, I * BM, U.h, U.b);
+          }
+          ++nI;
+          const int nT = n_col_tiles(p, I);
+          for (int J = 0; J < nT; ++J) {
+            const int st = nJ & 1;
+            const uint32_t par = ((nJ >> 1) & 1) ^ 1;
+            if (!(ok = mbar_wait(EMPTY_T(st), par, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_T(st), L::TILE);
+#pragma unroll
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_4d(base + L::XT_R + st * L::TILE + b * BOX, &U.seg->tm_t, FULL_T(st),
+                          b * 64, J * BN, U.h, U.b);
+            ++armsT[st];
+            if (!(ok = mbar_wait(EMPTY_S(st), par, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_S(st), L::TILE);
+#pragma unroll
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_4d(base + L::XS_R + st * L::TILE + b * BOX, &U.seg->tm_s, FULL_S(st),
+                          b * 64, J * BN, U.h, U.b);
+            ++armsS[st];
+            ++nJ;
+          }
+        }
+      }
+      // wait for the copies still in flight before the CTA may exit
+      if (nI) mbar_wait_drain(FULL_I, (nI - 1) & 1, kDrainNs);
+      for (int st = 0; st < 2; ++st) {
+        if (armsT[st]) mbar_wait_drain(FULL_T(st), (armsT[st] - 1) & 1, kDrainNs);
+        if (armsS[st]) mbar_wait_drain(FULL_S(st), (armsS[st] - 1) & 1, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 13) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t IDESC_GX = idesc_bf16_f32(BM, D, 0, 1);   // A = G (K-major), B = X (MN)
+      constexpr uint32_t IDESC_GTX = idesc_bf16_f32(BM, D, 1, 1);  // A = G^T (MN), B = X (MN)
+      uint32_t nI = 0, nJ = 0, ns = 0, ng = 0, nrb = 0;
+      bool ok = true, issued = false;
+      // gradient MMAs of the tile that used ring stage `st`; `first` starts dX_I
+      auto grad = [&](int st, bool first) -> bool {
+        if (!mbar_wait(G_FULL, ng & 1, wc, W_MMA_G_FULL)) return false;
+        if (!mbar_wait(P_EMPTY, (ng & 1) ^ 1, wc, W_MMA_P_EMPTY)) return false;
+        if (first && !mbar_wait(DXI_EMPTY, (nrb & 1) ^ 1, wc, W_MMA_DXI_EMPTY)) return false;
+        tc_fence_after();
+        const uint32_t g = base + L::G;
+        const uint32_t xsj = base + L::XS_R + st * L::TILE;
+        const uint32_t xsi = base + L::XS_I;
+        // dX_I += G X_s[J]: M = i, N = c, K = j
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k) {
+          const uint64_t ad = sw128_desc(g + (k >> 2) * BOX + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(xsj + k * 2048, BOX, 1024);
+          umma_bf16(tmem + T_DXI, ad, bd, IDESC_GX, (!first || k > 0) ? 1u : 0u);
+        }
+        // P = G^T X_s[I]: M = j, N = c, K = i
+#pragma unroll
+        for (int k = 0; k < BM / 16; ++k) {
+          const uint64_t ad = sw128_desc(g + k * 2048, BOX, 1024);
+          const uint64_t bd = sw128_desc(xsi + k * 2048, BOX, 1024);
+          umma_bf16(tmem + T_P, ad, bd, IDESC_GTX, k > 0 ? 1u : 0u);
+        }
+        umma_commit(G_EMPTY);
+        umma_commit(P_FULL);
+        umma_commit(EMPTY_S(st));
+        ++ng;
+        return true;
+      };
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        (void)u;
+        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+          const int I = pass_block(p, pp, pass);
+          if (!(ok = mbar_wait(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
+          const int nT = n_col_tiles(p, I);
+          int prev_st = -1;
+          for (int J = 0; J < nT; ++J) {
+            const int st = nJ & 1;
+            const uint32_t par = (nJ >> 1) & 1;
+            if (!(ok = mbar_wait(FULL_T(st), par, wc, W_MMA_FULL_J))) break;
+            if (!(ok = mbar_wait(FULL_S(st), par, wc, W_MMA_FULL_J))) break;
+            if (!(ok = mbar_wait(S_EMPTY, (ns & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
+            tc_fence_after();
+            issue_logits<D>(tmem + T_ST, base + L::XT_I, base + L::XT_R + st * L::TILE);
+            issue_logits<D>(tmem + T_SS, base + L::XS_I, base + L::XS_R + st * L::TILE);
+            issued = true;
+            umma_commit(EMPTY_T(st));
+            umma_commit(S_FULL);
+            ++ns;
+            ++nJ;
+            if (prev_st >= 0 && !(ok = grad(prev_st, J == 1))) break;
+            prev_st = st;
+          }
+          if (!ok) break;
+          if (!(ok = grad(prev_st, nT == 1))) break;
+          umma_commit(EMPTY_I);
+          umma_commit(DXI_FULL);
+          ++nI;
+          ++nrb;
+        }
+      }
+      if (issued) {
+        umma_commit(DRAIN);
+        mbar_wait_drain(DRAIN, 0, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 8) {
+    // ------------------------------------------------------- epilogue
+    const int q = warp - 8;
+    uint32_t np = 0, nrb = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      const Unit U = decode_unit(p, u);
+      float* dx = U.seg->dx + U.row0 * D;
+      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+        const int I = pass_block(p, pp, pass);
+        const int nT = n_col_tiles(p, I);
+        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        for (int J = 0; J < nT; ++J) {
+          ok = mbar_wait(P_FULL, np & 1, wc, W_EPI_P_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const int jrow = J * BN + q * 32 + lane;
+          float* dst = dx + static_cast<long long>(jrow) * D;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tmem_ld32(tmem + lane_addr + T_P + c * 32, v);
+            tmem_wait_ld();
+            if (c == D / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(P_EMPTY);
+            }
+            if (jrow < p.N) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                red_add_v4(dst + c * 32 + 4 * k, v[4 * k], v[4 * k + 1], v[4 * k + 2],
+                           v[4 * k + 3]);
+            }
+          }
+          ++np;
+        }
+        if (!ok) break;
+        ok = mbar_wait(DXI_FULL, nrb & 1, wc, W_EPI_DXI_FULL);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const int irow = I * BM + q * 32 + lane;
+        float* dst = dx + static_cast<long long>(irow) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(tmem + lane_addr + T_DXI + c * 32, v);
+          tmem_wait_ld();
+          if (c == D / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(DXI_EMPTY);
+          }
+          if (irow < p.N) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              red_add_v4(dst + c * 32 + 4 * k, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+          }
+        }
+        ++nrb;
+      }
+    }
+  } else {
+    // --------------------------------------------------- row warpgroups
+    const int q = warp & 3;
+    const int half = warp >> 2;
+    const int r = q * 32 + lane;
+    const float sl2 = p.sl2;
+    const uint32_t gsm = base + L::G + half * BOX + r * 128;
+    uint32_t ns = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      const Unit U = decode_unit(p, u);
+      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+        const int I = pass_block(p, pp, pass);
+        const int row = I * BM + r;
+        const bool rvalid = row < p.N;
+        float bt = 0.f, bs = 0.f, mul = 0.f;
+        if (rvalid) {
+          const float4 st4 = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + row];
+          bt = -st4.y * kLog2e;
+          bs = -st4.z * kLog2e;
+          const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(p.N);
+          mul = up * p.scale;   // the logit scale of dX_s is folded into G
+        }
+        const int lim = !rvalid ? -1 : (p.causal ? min(row, p.N - 1) : p.N - 1);
+        const int nT = n_col_tiles(p, I);
+        for (int J = 0; J < nT; ++J) {
+          ok = mbar_wait(S_FULL, ns & 1, wc, W_SM_S_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * 64;
+          const int col0 = J * BN + half * 64;
+          const bool need_mask = !rvalid || (col0 + 63 > lim);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float t[32], s[32];
+            tmem_ld32(ta + T_ST + c * 32, t);
+            tmem_ld32(ta + T_SS + c * 32, s);
+            tmem_wait_ld();
+            if (c == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(S_EMPTY);
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              float g0 = mul * (ex2_approx(fmaf(s[k], sl2, bs)) - ex2_approx(fmaf(t[k], sl2, bt)));
+              float g1 = mul * (ex2_approx(fmaf(s[k + 1], sl2, bs)) -
+                                ex2_approx(fmaf(t[k + 1], sl2, bt)));
+              if (need_mask) {
+                g0 = (col0 + c * 32 + k <= lim) ? g0 : 0.f;
+                g1 = (col0 + c * 32 + k + 1 <= lim) ? g1 : 0.f;
+              }
+              pk[k >> 1] = pack_bf16x2(g0, g1);
+            }
+            if (c == 0) {
+              // the G buffer is free once the previous tile's gradient MMAs completed
+              ok = mbar_wait(G_EMPTY, (ns & 1) ^ 1, wc, W_SM_G_EMPTY);
+              ok = __all_sync(0xffffffffu, ok);
+              if (!ok) break;
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int cc = c * 4 + q4;  // 16-byte chunk within the 128-byte row
+              st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[4 * q4], pk[4 * q4 + 1],
+                           pk[4 * q4 + 2], pk[4 * q4 + 3]);
+            }
+          }
+          if (!ok) break;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(G_FULL);
+          ++ns;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------ launchers
+template <int D>
+static cudaError_t launch_fwd(const TcParams& p, int grid, cudaStream_t stream) {
+  auto k = relkl_fwd_tc_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       FwdSmem<D>::ALLOC);
+  if (e != cudaSuccess) return e;
+  k<<<grid, FWD_THREADS, FwdSmem<D>::ALLOC, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_bwd(const TcParams& p, int grid, cudaStream_t stream) {
+  auto k = relkl_bwd_tc_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       BwdSmem<D>::ALLOC);
+  if (e != cudaSuccess) return e;
+  k<<<grid, BWD_THREADS, BwdSmem<D>::ALLOC, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t tc_launch_fwd(const TcParams& p, int d, int grid, cudaStream_t stream) {
+  return d == 64 ? launch_fwd<64>(p, grid, stream) : launch_fwd<128>(p, grid, stream);
+}
+
+cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t stream) {
+  return d == 64 ? launch_bwd<64>(p, grid, stream) : launch_bwd<128>(p, grid, stream);
+}
+
+size_t tc_smem_bytes(int d, int is_bwd) {
+  if (is_bwd) return d == 64 ? BwdSmem<64>::ALLOC : BwdSmem<128>::ALLOC;
+  return d == 64 ? FwdSmem<64>::ALLOC : FwdSmem<128>::ALLOC;
+}
+
+}  // namespace relkl

@@ -1,0 +1,213 @@
+"""PyTorch-facing binding of librelkl.so, with the C ABI's names.
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current CUDA stream.  There is
+no CPU fallback; calls raise if the library is missing or a tensor is not on a
+CUDA device.
+
+Layout contract (include/relkl.h): teacher and student are [B, H, N, d]
+tensors with a contiguous last dimension; kl is [B, H, N] float32, stats is
+[B, H, N, 4] float32 (m, lse_t, lse_s, w) and dX_s is [B, H, N, d] float32.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import torch
+
+from . import _abi
+from ._abi import check, relkl_desc
+
+__all__ = ["relkl_fwd", "relkl_bwd", "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_workspace_bytes",
+           "relkl_workspace_init", "relkl_get_device_error", "relkl_set_wait_timeout_ns",
+           "relkl_path_for", "workspace", "make_desc", "relation_kl", "RelationKL"]
+
+_DTYPES = {torch.bfloat16: _abi.RELKL_BF16, torch.float32: _abi.RELKL_FP32}
+
+
+def make_desc(x: torch.Tensor, causal: bool = True, scale: float = 0.0) -> relkl_desc:
+    if x.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    if x.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {x.dtype}")
+    d = relkl_desc()
+    d.B, d.H, d.N, d.d = (int(v) for v in x.shape)
+    for i in range(3):          # a dimension of extent 1 has no meaningful stride
+        d.stride[i] = int(x.stride(i)) if x.shape[i] != 1 else 0
+    d.stride[3] = 1 if (x.shape[3] == 1 or x.stride(3) == 1) else int(x.stride(3))
+    d.dtype = _DTYPES[x.dtype]
+    d.causal = 1 if causal else 0
+    d.scale = float(scale)
+    d.reserved = 0
+    return d
+
+
+def _stream(device: torch.device, stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _cuda(t: torch.Tensor, name: str) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+
+
+_WS: Dict[int, torch.Tensor] = {}
+
+
+def relkl_workspace_bytes() -> int:
+    return int(_abi.lib().relkl_workspace_bytes())
+
+
+def relkl_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    check(_abi.lib().relkl_workspace_init(_ptr(ws), ws.numel() * ws.element_size(),
+                                          _stream(ws.device, stream)), "relkl_workspace_init")
+
+
+def workspace(device=None) -> torch.Tensor:
+    """A zeroed per-device workspace (the device error record), cached."""
+    device = torch.device(device or "cuda")
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    ws = _WS.get(idx)
+    if ws is None:
+        ws = torch.empty(relkl_workspace_bytes(), dtype=torch.uint8, device=f"cuda:{idx}")
+        relkl_workspace_init(ws)
+        _WS[idx] = ws
+    return ws
+
+
+def relkl_path_for(x: torch.Tensor, causal: bool = True, scale: float = 0.0) -> int:
+    d = make_desc(x, causal, scale)
+    return int(_abi.lib().relkl_path_for(ctypes.byref(d)))
+
+
+def _arr(vals, ctype=ctypes.c_void_p):
+    return (ctype * len(vals))(*[v if v is not None else None for v in vals])
+
+
+def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bool = True,
+                  scale: float = 0.0, *, out: Optional[Sequence[Tuple[torch.Tensor, torch.Tensor]]] = None,
+                  ws: Optional[torch.Tensor] = None, stream=None):
+    """Forward over 1..3 relations in one launch.  Returns [(kl, stats)] per relation."""
+    n = len(pairs)
+    if not 1 <= n <= 3:
+        raise ValueError("1 to 3 relations per call")
+    dev = pairs[0][0].device
+    descs = (relkl_desc * n)()
+    outs = []
+    for r, (xt, xs) in enumerate(pairs):
+        _cuda(xt, "x_t")
+        _cuda(xs, "x_s")
+        if xt.shape != xs.shape or xt.stride() != xs.stride() or xt.dtype != xs.dtype:
+            raise ValueError("teacher and student must share shape, strides and dtype")
+        descs[r] = make_desc(xt, causal, scale)
+        B, H, N, _ = xt.shape
+        if out is not None:
+            kl, st = out[r]
+        else:
+            kl = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+            st = torch.empty((B, H, N, 4), dtype=torch.float32, device=dev)
+        outs.append((kl, st))
+    ws = workspace(dev) if ws is None else ws
+    code = _abi.lib().relkl_fwd_qkv(
+        n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
+        _arr([_ptr(o[0]) for o in outs]), _arr([_ptr(o[1]) for o in outs]),
+        _ptr(ws), ws.numel(), _stream(dev, stream))
+    check(code, "relkl_fwd_qkv")
+    return outs
+
+
+def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Sequence[torch.Tensor],
+                  dkl: Optional[Sequence[Optional[torch.Tensor]]] = None, causal: bool = True,
+                  scale: float = 0.0, *, out: Optional[Sequence[torch.Tensor]] = None,
+                  ws: Optional[torch.Tensor] = None, stream=None) -> List[torch.Tensor]:
+    """Backward over 1..3 relations in one launch.  Returns dX_s per relation (float32)."""
+    n = len(pairs)
+    if not 1 <= n <= 3 or len(stats) != n:
+        raise ValueError("1 to 3 relations per call, with one stats tensor each")
+    dev = pairs[0][0].device
+    descs = (relkl_desc * n)()
+    dxs = []
+    for r, (xt, xs) in enumerate(pairs):
+        _cuda(xt, "x_t")
+        _cuda(xs, "x_s")
+        if xt.shape != xs.shape or xt.stride() != xs.stride() or xt.dtype != xs.dtype:
+            raise ValueError("teacher and student must share shape, strides and dtype")
+        descs[r] = make_desc(xt, causal, scale)
+        if not stats[r].is_contiguous() or stats[r].dtype != torch.float32:
+            raise ValueError("stats must be contiguous float32 [B, H, N, 4]")
+        if dkl is not None and dkl[r] is not None and (not dkl[r].is_contiguous()
+                                                       or dkl[r].dtype != torch.float32):
+            raise ValueError("dkl must be contiguous float32 [B, H, N]")
+        dx = out[r] if out is not None else torch.empty(xs.shape, dtype=torch.float32, device=dev)
+        if not dx.is_contiguous() or dx.dtype != torch.float32:
+            raise ValueError("dx_s must be contiguous float32")
+        dxs.append(dx)
+    ws = workspace(dev) if ws is None else ws
+    dkl_arr = None if dkl is None else _arr([_ptr(g) for g in dkl])
+    code = _abi.lib().relkl_bwd_qkv(
+        n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
+        _arr([_ptr(s) for s in stats]), dkl_arr, _arr([_ptr(d) for d in dxs]),
+        _ptr(ws), ws.numel(), _stream(dev, stream))
+    check(code, "relkl_bwd_qkv")
+    return dxs
+
+
+def relkl_fwd(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True, scale: float = 0.0, *,
+              kl: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
+              ws: Optional[torch.Tensor] = None, stream=None):
+    """Per-row KL [B,H,N] and statistics [B,H,N,4] of one relation."""
+    out = None if kl is None else [(kl, stats)]
+    return relkl_fwd_qkv([(x_t, x_s)], causal, scale, out=out, ws=ws, stream=stream)[0]
+
+
+def relkl_bwd(x_t: torch.Tensor, x_s: torch.Tensor, stats: torch.Tensor,
+              dkl: Optional[torch.Tensor] = None, causal: bool = True, scale: float = 0.0, *,
+              dx_s: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """dL/dX_s (float32) with L = sum_i dkl_i kl_i (dkl=None: 1/N per row)."""
+    return relkl_bwd_qkv([(x_t, x_s)], [stats], None if dkl is None else [dkl], causal, scale,
+                         out=None if dx_s is None else [dx_s], ws=ws, stream=stream)[0]
+
+
+def relkl_get_device_error(ws: Optional[torch.Tensor] = None, stream=None) -> Tuple[int, int]:
+    """Synchronise the stream and read the workspace record: (status, wait site)."""
+    ws = workspace() if ws is None else ws
+    where = ctypes.c_uint32(0)
+    code = _abi.lib().relkl_get_device_error(_ptr(ws), _stream(ws.device, stream),
+                                             ctypes.byref(where))
+    return int(code), int(where.value)
+
+
+def relkl_set_wait_timeout_ns(ns: int) -> int:
+    return int(_abi.lib().relkl_set_wait_timeout_ns(int(ns)))
+
+
+class RelationKL(torch.autograd.Function):
+    """kl rows of one relation; backward runs relkl_bwd (teacher is frozen)."""
+
+    @staticmethod
+    def forward(ctx, x_t, x_s, causal=True, scale=0.0):
+        kl, stats = relkl_fwd(x_t.detach(), x_s.detach(), causal, scale)
+        ctx.save_for_backward(x_t, x_s, stats)
+        ctx.causal, ctx.scale = causal, scale
+        return kl
+
+    @staticmethod
+    def backward(ctx, dkl):
+        x_t, x_s, stats = ctx.saved_tensors
+        dx = relkl_bwd(x_t.detach(), x_s.detach(), stats, dkl.contiguous().float(), ctx.causal,
+                       ctx.scale)
+        return None, dx, None, None
+
+
+def relation_kl(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,
+                scale: float = 0.0) -> torch.Tensor:
+    """Differentiable per-row KL(R_t || R_s) of one relation, shape [B, H, N]."""
+    return RelationKL.apply(x_t, x_s, causal, scale)

@@ -1,0 +1,375 @@
+"""Benchmark of the relation-KL hot path: fused Q/K/V forward + backward.
+
+One step = relkl_fwd_qkv + relkl_bwd_qkv over every (batch, head, relation)
+unit of the workload (default: the 32K extended-context training shape,
+B=1, H=32, N=32768, d=128, bf16, causal, Q/K/V -> 96 units).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference ...   # the float64 CPU oracle, host cores
+
+Prints ONE JSON line on rank 0.  ``value`` is algorithmic fwd+bwd TFLOP/s of
+the whole job (12*d*E flops per unit, E = N(N+1)/2 causal entries), device
+timed with CUDA events between barriers, max over ranks.  Under torchrun each
+rank runs its own replica of the workload (independent units, no collective on
+the data path): weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workload  # noqa: E402
+
+METRIC = "relation-KL fwd+bwd TFLOP/s & tokens/s at N=32K,d=128; % of BF16 tensor peak"
+L2_BYTES = 126 * 2**20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def flops(w: workload.Workload):
+    E = w.N * (w.N + 1) / 2 if w.causal else float(w.N) ** 2
+    per_unit_fwd, per_unit_bwd = 4.0 * w.d * E, 8.0 * w.d * E
+    return per_unit_fwd * w.n_units, per_unit_bwd * w.n_units
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def traffic_record(kernel: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it matches the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "attention_relation_kl_b200", "csrc", "relkl_tc.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return rec.get("bytes_per_launch") if rec.get("source_sha256") == h else None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            self.path = f"/tmp/relkl_clocks_{os.getpid()}.csv"
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle arm
+
+def oracle_sample(w: workload.Workload, n_prefix: int, n_units: int, seed_inputs=None):
+    """Time the float64 oracle (fwd + bwd) on the causal prefix [0, n_prefix) of the
+    first n_units units of the workload: exactly the relation-KL of those rows."""
+    from oracle import dense
+    x = seed_inputs if seed_inputs is not None else workload.generate(
+        workload.Workload(**{**w.__dict__, "B": 1, "H": 1, "H_kv": 1}))
+    units = [(r, 0, 0) for r in w.relations][:n_units]
+    E = n_prefix * (n_prefix + 1) / 2 if w.causal else float(n_prefix) ** 2
+    t0 = time.perf_counter()
+    for rel, b, h in units:
+        xt = x[rel][0][b, h, :n_prefix]
+        xs = x[rel][1][b, h, :n_prefix]
+        dense.fwd_unit(xt, xs, w.causal)
+        dense.bwd_unit(xt, xs, None, w.causal)
+    dt = time.perf_counter() - t0
+    fl = 12.0 * w.d * E * len(units)
+    return fl / dt / 1e12, dt, units
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w: workload.Workload, budget_s: float = 20.0):
+    # grow the prefix until one fwd+bwd pass over 3 units takes ~budget_s
+    n = 1024
+    tf, dt, units = oracle_sample(w, n, 3)
+    while dt < budget_s / 4 and n * 2 <= w.N:
+        n *= 2
+        tf, dt, units = oracle_sample(w, n, 3)
+    return {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"float64 oracle fwd+bwd on the causal row prefix [0,{n}) of units "
+                      f"{[u[0] + str(u[2]) for u in units]} of {w.name} "
+                      f"({dt:.1f} s); TFLOP/s counted as 12*d*E per unit",
+            "seconds": dt}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x = workload.generate(workload.Workload(**{**w.__dict__, "B": 1, "H": 1, "H_kv": 1}))
+    n_prefix = args.ref_prefix
+    for _ in range(args.warmup):
+        oracle_sample(w, n_prefix, 1, x)
+    times = []
+    for _ in range(args.steps):
+        tf, dt, units = oracle_sample(w, n_prefix, len(w.relations), x)
+        times.append(dt)
+    E = n_prefix * (n_prefix + 1) / 2
+    fl = 12.0 * w.d * E * len(w.relations)
+    value = fl * args.steps / sum(times) / 1e12
+    sample = (f"float64 oracle fwd+bwd per step on the causal prefix [0,{n_prefix}) of one "
+              f"head of each relation {list(w.relations)} of {w.name}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N,
+                       "d": w.d, "relations": "".join(w.relations), "causal": w.causal,
+                       "sample_prefix": n_prefix},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="ext_h32_n32k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--ref-prefix", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = workload.get_config(args.config)
+
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch.distributed as dist
+    import attention_relation_kl_b200 as rk
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # inputs: this rank's replica (seed offset by rank), resident in HBM
+    wr = workload.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
+    t_gen = time.perf_counter()
+    x = workload.generate(wr)
+    t_gen = time.perf_counter() - t_gen
+    host = {r: (x[r][0].pin_memory(), x[r][1].pin_memory()) for r in w.relations}
+    pairs = [(host[r][0].to(dev), host[r][1].to(dev)) for r in w.relations]
+    in_bytes = sum(a.numel() * a.element_size() * 2 for a, _ in pairs)
+    ws = rk.workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_alloc = torch.cuda.memory_allocated(dev)
+
+    outs = rk.relkl_fwd_qkv(pairs, w.causal, ws=ws)
+    dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, ws=ws)
+    torch.cuda.synchronize()
+    out_dx_bytes = sum(d.numel() * 4 for d in dxs)
+    stats_bytes = sum(o[0].numel() * 4 + o[1].numel() * 4 for o in outs)
+
+    def step():
+        rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
+        rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    code, where = rk.relkl_get_device_error(ws)
+    if code != 0:
+        raise SystemExit(f"device wait ran out during warm-up (site {where})")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
+        ev[i][1].record(stream)
+        rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    bwd_ms = [b.elapsed_time(c) for _, b, c in ev]
+    code, where = rk.relkl_get_device_error(ws)
+    if code != 0:
+        raise SystemExit(f"device wait ran out in the timed region (site {where})")
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    peak_alloc = torch.cuda.max_memory_allocated(dev)
+
+    # end to end through the public API with host buffers
+    e2e_ms = None
+    h2d = sum(host[r][0].numel() * host[r][0].element_size() * 2 for r in w.relations)
+    host_dx = [torch.empty(d.shape, dtype=torch.float32, pin_memory=True) for d in dxs]
+    host_kl = [torch.empty(o[0].shape, dtype=torch.float32, pin_memory=True) for o in outs]
+    d2h = sum(h.numel() * 4 for h in host_dx) + sum(h.numel() * 4 for h in host_kl)
+    if args.e2e_steps > 0:
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for (gt, gs), r in zip(pairs, w.relations):
+                gt.copy_(host[r][0], non_blocking=True)
+                gs.copy_(host[r][1], non_blocking=True)
+            o = rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
+            dd = rk.relkl_bwd_qkv(pairs, [q[1] for q in o], None, w.causal, out=dxs, ws=ws)
+            for hk, (kl, _) in zip(host_kl, o):
+                hk.copy_(kl, non_blocking=True)
+            for hd, dv in zip(host_dx, dd):
+                hd.copy_(dv, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+
+    fl_fwd, fl_bwd = flops(w)
+    total_fl = (fl_fwd + fl_bwd) * world
+    ms_step = ms / args.steps
+    value = total_fl / (ms_step * 1e-3) / 1e12
+    tokens = w.B * w.N * world / (ms_step * 1e-3)
+
+    peaks, peak_src = load_peaks()
+    peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    bwd_avg = sum(bwd_ms) / len(bwd_ms)
+    fwd_avg = sum(fwd_ms) / len(fwd_ms)
+    achieved = fl_bwd / (bwd_avg * 1e-3) / 1e12
+    traffic = traffic_record("relkl_bwd_tc_kernel")
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(w)
+        result = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
+                       "relations": "".join(w.relations), "causal": w.causal,
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": f"inputs {in_bytes / 1e9:.2f} GB > L2 126 MB (no flush)"},
+            "tokens_per_s": tokens,
+            "pct_bf16_peak": 100.0 * value / (peak_tf * world),
+            "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
+            "fwd_tflops": fl_fwd / (fwd_avg * 1e-3) / 1e12,
+            "bwd_tflops": fl_bwd / (bwd_avg * 1e-3) / 1e12,
+            "roofline": {"kernel": "relkl_bwd_tc_kernel", "bound": "tensor", "achieved": achieved,
+                         "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                         "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                         "achieved_note": "8*d*E flops per unit x units per launch / CUDA-event time "
+                                          "of the relkl_bwd_qkv call (dX zeroing included)"},
+            "e2e": {"value": None if e2e_ms is None else total_fl / (e2e_ms * 1e-3) / 1e12,
+                    "unit": "TFLOP/s", "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * (2 + len(w.relations)),
+            "memory": {"peak_allocated_bytes": peak_alloc, "inputs_bytes": in_bytes,
+                       "dx_bytes": out_dx_bytes, "row_stats_bytes": stats_bytes,
+                       "extra_bytes": peak_alloc - base_alloc - out_dx_bytes,
+                       "workspace_bytes": rk.relkl_workspace_bytes()},
+            "clocks": clk,
+            "input_generation_s": t_gen,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,149 @@
+/*
+ * relkl.h -- C ABI of librelkl.so: the linear-memory relation-distillation KL
+ * loss of LinearARD and its gradient, on NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  LinearARD (arXiv 2604.00004; pith.science verdict page,
+ * field pith_extraction.key_machinery, repeated in core_discovery; the
+ * abstract on the mlsanity.com index page) distils, for every head and for
+ * X in {Q, K, V}, the row-wise distributions of the masked self-relation
+ *
+ *     Z_m = X_m X_m^T * scale + M,   R_m = softmax_rows(Z_m),  m in {t, s},
+ *
+ * of a frozen teacher (t) into a RoPE-scaled student (s) by the forward KL
+ *
+ *     kl_i = KL(R_t(i,:) || R_s(i,:)),   L = (1/n) sum_i kl_i,
+ *
+ * and backpropagates through the identity dL/dZ_s(i,j) = (R_s - R_t)(i,j)/n.
+ * With an upstream gradient dkl_i per row, G(i,j) = dkl_i (R_s - R_t)(i,j) on
+ * allowed entries and, because X_s appears on both sides of Z_s,
+ *
+ *     dX_s = scale * (G + G^T) X_s.
+ *
+ * M is the causal mask (column j allowed for row i iff j <= i) when
+ * `causal` is set, and no mask otherwise; the pages name M without defining
+ * it.  No N x N matrix is ever stored: the forward keeps O(N) row statistics
+ * and the backward recomputes the logit tiles (the pages' two-phase scheme).
+ *
+ * A "unit" is one (batch b, head h) slice of one relation: an [N, d] teacher
+ * matrix and the matching student matrix.  Units are independent.
+ *
+ * Conventions for every entry point below:
+ *  - All tensor pointers are DEVICE pointers, owned by the caller, and must
+ *    stay valid until the work queued on `stream` has finished.  The library
+ *    allocates no device or host memory and keeps no pointer after a call.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    only enqueue work on it and return; nothing synchronises except
+ *    relkl_get_device_error().
+ *  - Arguments are validated before anything is enqueued; on any error code
+ *    other than RELKL_OK nothing was enqueued, except RELKL_ERR_CUDA, which
+ *    reports a failed launch (see relkl_last_cuda_error()).
+ *  - Row statistics and gradients are float32.  Teacher and student inputs
+ *    are bf16 (tensor-core path, d in {64, 128}) or float32 (CUDA-core path,
+ *    1 <= d <= 128).
+ */
+#ifndef RELKL_H
+#define RELKL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RELKL_OK = 0,
+  RELKL_ERR_INVALID = 1,      /* null pointer, bad shape, stride or alignment      */
+  RELKL_ERR_UNSUPPORTED = 2,  /* well-formed but not provided (e.g. bf16 with d=96) */
+  RELKL_ERR_CUDA = 3,         /* a CUDA runtime or driver call failed               */
+  RELKL_ERR_WORKSPACE = 4,    /* workspace missing, misaligned or too small          */
+  RELKL_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out (device record)  */
+} relkl_status;
+
+typedef enum { RELKL_BF16 = 0, RELKL_FP32 = 1 } relkl_dtype;
+
+/* Shape of one relation's teacher AND student tensors (both use it).
+ * Logical shape [B, H, N, d]; element (b,h,n,k) lives at
+ *   base + b*stride[0] + h*stride[1] + n*stride[2] + k      (elements).
+ * stride[3] must be 1.  For the bf16 path the base address and stride[0..2]
+ * (in bytes) must be multiples of 16 (a TMA requirement).                    */
+typedef struct {
+  int32_t B, H, N, d;
+  int64_t stride[4];
+  int32_t dtype;     /* relkl_dtype                                         */
+  int32_t causal;    /* 1: row i sees columns j <= i; 0: every column       */
+  float scale;       /* logit scale; 0 means 1/sqrt(d)                      */
+  int32_t reserved;  /* must be 0                                           */
+} relkl_desc;
+
+/* Bytes of device workspace a call needs (for every entry point, any desc):
+ * a 256-byte, 256-byte-aligned record that the kernels use to report a
+ * bounded wait that ran out.  Zero it once after allocation
+ * (relkl_workspace_init); calls never clear it, so a reported error sticks
+ * until the caller clears it again.                                          */
+size_t relkl_workspace_bytes(void);
+relkl_status relkl_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Forward (Phase 1 on the pages: per-row statistics, O(N) memory).
+ *   x_t, x_s : teacher / student, layout `desc`.
+ *   kl       : float [B, H, N] contiguous, out: kl_i per row.
+ *   stats    : float [B, H, N, 4] contiguous, out, per row
+ *              (m, lse_t, lse_s, w): m = max_j max(Z_t, Z_s)(i,j) over allowed
+ *              j, lse_m = log sum_j exp Z_m(i,j), w = sum_j R_t (Z_t - Z_s)(i,j).
+ *              kl_i = w_i + lse_s(i) - lse_t(i).  Needed by relkl_bwd.      */
+relkl_status relkl_fwd(const relkl_desc* desc, const void* x_t, const void* x_s,
+                       float* kl, float* stats, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Backward (Phase 2 on the pages: recompute the logit tiles, rebuild R_t and
+ * R_s from the stored LSEs, form G and stream it into dX_s).
+ *   stats    : the forward's statistics for the same inputs.
+ *   dkl      : float [B, H, N] contiguous upstream gradient of kl, or NULL for
+ *              1/N on every row (the gradient of L = (1/N) sum_i kl_i).
+ *   dx_s     : float [B, H, N, d] contiguous, out: overwritten with dL/dX_s.
+ * The teacher is frozen and gets no gradient.  dx_s is accumulated with
+ * float32 atomics, so its last bits depend on scheduling.                   */
+relkl_status relkl_bwd(const relkl_desc* desc, const void* x_t, const void* x_s,
+                       const float* stats, const float* dkl, float* dx_s,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Several relations (Q, K, V of one layer; GQA gives K and V fewer heads)
+ * in ONE persistent launch.  n_rel in 1..3; descs[r] describes relation r.
+ * All descs must share N, d, dtype, causal and scale; B and H may differ.
+ * Arrays are indexed by relation, with the meaning of relkl_fwd / relkl_bwd.
+ * dkl may be NULL (all relations use 1/N) or an array whose entries may be NULL. */
+relkl_status relkl_fwd_qkv(int32_t n_rel, const relkl_desc* descs,
+                           const void* const* x_t, const void* const* x_s,
+                           float* const* kl, float* const* stats,
+                           void* ws, size_t ws_bytes, void* stream);
+relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs,
+                           const void* const* x_t, const void* const* x_s,
+                           const float* const* stats, const float* const* dkl,
+                           float* const* dx_s, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Synchronises `stream`, then reads the workspace record.  Returns RELKL_OK
+ * or RELKL_ERR_TIMEOUT; *where (if not NULL) receives the code of the wait
+ * that ran out (0 when none).                                                */
+relkl_status relkl_get_device_error(const void* ws, void* stream, uint32_t* where);
+
+/* Test hook: bound every device-side wait of later launches from this
+ * process by `ns` nanoseconds (default 2e9).  0 makes any wait that is not
+ * satisfied at once run out, which exercises the timeout path without a
+ * hang.  Returns the previous value.                                         */
+uint64_t relkl_set_wait_timeout_ns(uint64_t ns);
+
+/* Human-readable name of a status code (static string).                     */
+const char* relkl_status_string(relkl_status s);
+
+/* The cudaError_t of the last failing CUDA call in this thread (0 if none). */
+int32_t relkl_last_cuda_error(void);
+
+/* Which kernel family a desc would run: 1 = tcgen05 tensor-core path,
+ * 2 = CUDA-core float32 path, 0 = unsupported.  Validation-free.            */
+int32_t relkl_path_for(const relkl_desc* desc);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RELKL_H */

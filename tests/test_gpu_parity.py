@@ -1,0 +1,203 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs, element by element.
+
+Small cases span several 128-row tiles with a ragged tail; the workload-sized
+cases run the fused Q/K/V launch the bench times and compare sampled units
+(and, for dX, sampled rows) that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import attention_relation_kl_b200 as rk
+import workload
+from oracle import dense
+from parity import DX_TOL_BF16, DX_TOL_FP32, assert_dx, assert_kl, assert_stats, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    rk.relkl_set_wait_timeout_ns(2_000_000_000)
+
+
+def _device_ok():
+    code, where = rk.relkl_get_device_error()
+    assert code == 0, f"device wait ran out at site {where}"
+
+
+def check_full(xt, xs, causal=True, dkl=None, dx_tol=DX_TOL_BF16, path=None):
+    """Run fwd+bwd on the GPU and compare every output with the oracle."""
+    dev = "cuda"
+    gt, gs = xt.to(dev), xs.to(dev)
+    if path is not None:
+        assert rk.relkl_path_for(gt, causal) == path
+    kl, st = rk.relkl_fwd(gt, gs, causal)
+    dx = rk.relkl_bwd(gt, gs, st, None if dkl is None else dkl.to(dev), causal)
+    torch.cuda.synchronize()
+    _device_ok()
+    ref = dense.fwd(xt, xs, causal)
+    assert_kl(to_np(kl), ref["kl"])
+    assert_stats(to_np(st), ref)
+    assert_dx(to_np(dx), dense.bwd(xt, xs, dkl, causal), dx_tol)
+
+
+def q_inputs(B, H, N, d, dtype="bf16", seed=0, causal=True, pi=4.0):
+    w = workload.tiny_custom(N=N, d=d, dtype=dtype, seed=seed, pi_factor=pi, causal=causal, B=B, H=H)
+    return workload.generate(w)["q"]
+
+
+# ----------------------------------------------------------- small shapes
+
+def test_tc_single_tile():
+    xt, xs = workload.gaussian_pair((1, 1, 128, 128), seed=1, noise=0.3, dtype=torch.bfloat16)
+    check_full(xt, xs, path=1)
+
+
+@pytest.mark.parametrize("N,d,causal,B,H", [
+    (1, 128, True, 1, 1), (2, 64, True, 1, 1), (127, 128, True, 1, 2), (129, 128, True, 2, 1),
+    (300, 64, True, 1, 2), (300, 128, False, 1, 2), (513, 64, False, 1, 1), (1000, 128, True, 1, 1),
+])
+def test_tc_shapes_rope_pi(N, d, causal, B, H):
+    xt, xs = q_inputs(B, H, N, d, seed=N + d, causal=causal)
+    check_full(xt, xs, causal=causal, path=1)
+
+
+def test_tc_value_relation_small_kl():
+    # V-like: student = teacher + small noise, KL ~ 1e-3 per row
+    xt, xs = workload.gaussian_pair((1, 2, 640, 128), seed=5, noise=0.05, dtype=torch.bfloat16)
+    check_full(xt, xs)
+
+
+def test_simt_fp32_tiny_config():
+    w = workload.CONFIGS["tiny_fp32_n256"]
+    xt, xs = workload.generate(w)["q"]
+    check_full(xt, xs, dx_tol=DX_TOL_FP32, path=2)
+
+
+def test_simt_bf16_unsupported_head_dim():
+    xt, xs = q_inputs(1, 2, 200, 96, seed=3)
+    check_full(xt, xs, dx_tol=DX_TOL_FP32, path=2)
+
+
+def test_upstream_gradient():
+    xt, xs = q_inputs(2, 2, 260, 128, seed=11)
+    dkl = torch.randn(2, 2, 260, generator=torch.Generator().manual_seed(2)) / 260
+    check_full(xt, xs, dkl=dkl)
+    xt32, xs32 = q_inputs(1, 1, 70, 64, dtype="fp32", seed=12)
+    check_full(xt32, xs32, dkl=torch.linspace(-1, 1, 70).reshape(1, 1, 70), dx_tol=DX_TOL_FP32)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_identical_inputs_give_exact_zero(dtype):
+    xt, _ = q_inputs(1, 2, 333, 128 if dtype == "bf16" else 64, dtype=dtype, seed=4)
+    g = xt.cuda()
+    kl, st = rk.relkl_fwd(g, g.clone())
+    dx = rk.relkl_bwd(g, g.clone(), st)
+    torch.cuda.synchronize()
+    assert torch.all(kl == 0) and torch.all(dx == 0)
+
+
+def test_strided_inputs():
+    # [B, N, H, d] storage (a fused projection output) viewed as [B, H, N, d]
+    gen = torch.Generator().manual_seed(9)
+    base_t = torch.randn(1, 384, 3, 128, generator=gen).to(torch.bfloat16)
+    base_s = (base_t.float() + 0.2 * torch.randn(1, 384, 3, 128, generator=gen)).to(torch.bfloat16)
+    xt, xs = base_t.permute(0, 2, 1, 3), base_s.permute(0, 2, 1, 3)
+    assert not xt.is_contiguous()
+    kl, st = rk.relkl_fwd(base_t.cuda().permute(0, 2, 1, 3), base_s.cuda().permute(0, 2, 1, 3))
+    dx = rk.relkl_bwd(base_t.cuda().permute(0, 2, 1, 3), base_s.cuda().permute(0, 2, 1, 3), st)
+    torch.cuda.synchronize()
+    ref = dense.fwd(xt, xs)
+    assert_kl(to_np(kl), ref["kl"])
+    assert_dx(to_np(dx), dense.bwd(xt, xs), DX_TOL_BF16)
+
+
+def test_fused_qkv_gqa_small():
+    g = workload.Workload("gqa_small", B=2, H=4, H_kv=2, N=300, d=128, dtype="bf16", causal=True,
+                          relations=("q", "k", "v"), rope_base=5e5, pi_factor=4.0, v_noise=0.05,
+                          seed=21)
+    x = workload.generate(g)
+    pairs = [(x[r][0].cuda(), x[r][1].cuda()) for r in "qkv"]
+    outs = rk.relkl_fwd_qkv(pairs)
+    dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs])
+    torch.cuda.synchronize()
+    _device_ok()
+    for r, (kl, st), dx in zip("qkv", outs, dxs):
+        ref = dense.fwd(*x[r])
+        assert_kl(to_np(kl), ref["kl"], what=f"kl[{r}]")
+        assert_stats(to_np(st), ref)
+        assert_dx(to_np(dx), dense.bwd(*x[r]), DX_TOL_BF16)
+
+
+def test_forward_is_deterministic():
+    xt, xs = q_inputs(1, 4, 700, 128, seed=13)
+    gt, gs = xt.cuda(), xs.cuda()
+    a = rk.relkl_fwd(gt, gs)
+    b = rk.relkl_fwd(gt, gs)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_autograd_wrapper():
+    xt, xs = q_inputs(1, 2, 200, 128, seed=17)
+    gt = xt.cuda()
+    gs = xs.cuda().requires_grad_(True)
+    kl = rk.relation_kl(gt, gs)
+    kl.mean().backward()
+    torch.cuda.synchronize()
+    # mean over B*H*N rows: dkl = 1/(B*H*N) per row
+    dkl = torch.full((1, 2, 200), 1.0 / (2 * 200))
+    assert_dx(to_np(gs.grad), dense.bwd(xt, xs, dkl), DX_TOL_BF16)
+
+
+# ------------------------------------------------------ workload sizes
+
+SAMPLE_ROWS = (0, 1, 127, 128, 129)
+
+
+def _sampled(w: workload.Workload, units, dx_units, n_dx_rows=6):
+    """Fused Q/K/V launch of the whole workload; oracle on sampled units."""
+    x = workload.generate(w)
+    pairs = [(x[r][0].cuda(), x[r][1].cuda()) for r in w.relations]
+    outs = rk.relkl_fwd_qkv(pairs, w.causal)
+    dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal)
+    torch.cuda.synchronize()
+    _device_ok()
+    rel_idx = {r: i for i, r in enumerate(w.relations)}
+    N = w.N
+    rows = sorted(set([r for r in SAMPLE_ROWS if r < N] + [N // 2, N - 129, N - 2, N - 1]))
+    for (rel, b, h) in units:
+        xt, xs = x[rel][0][b, h], x[rel][1][b, h]
+        kl, st = outs[rel_idx[rel]]
+        full = (rel, b, h) in dx_units
+        ref = dense.fwd_unit(xt, xs, w.causal) if full else dense.fwd_rows(xt, xs, rows, w.causal)
+        sel = slice(None) if full else rows
+        assert_kl(to_np(kl[b, h])[sel], ref["kl"], what=f"kl[{rel},{b},{h}]")
+        assert_stats(to_np(st[b, h])[sel], ref)
+        if full:
+            dx_rows = rows[:n_dx_rows] + rows[-2:]
+            ref_dx = dense.bwd_rows(xt, xs, dx_rows, causal=w.causal, lse=ref)
+            got = to_np(dxs[rel_idx[rel]][b, h])[dx_rows]
+            assert_dx(got, ref_dx, DX_TOL_BF16)
+
+
+def test_config_llama2_h32_n4k():
+    w = workload.CONFIGS["llama2_h32_n4k"]
+    units = [("q", 0, 0), ("q", 0, 31), ("k", 0, 7), ("v", 0, 0), ("v", 0, 31)]
+    _sampled(w, units, dx_units=set(units))
+
+
+def test_config_gqa_llama3_n16k():
+    w = workload.CONFIGS["gqa_llama3_n16k"]
+    units = [("q", 1, 31), ("k", 0, 3), ("v", 1, 7)]
+    _sampled(w, units, dx_units={("v", 1, 7)})
+
+
+def test_config_ext_h32_n32k():
+    w = workload.CONFIGS["ext_h32_n32k"]
+    units = [("q", 0, 0), ("k", 0, 17), ("v", 0, 31)]
+    _sampled(w, units, dx_units={("q", 0, 0)})
