@@ -7,10 +7,10 @@ Compute runs in librelkl.so (tcgen05/TMA kernels); this package only marshals
 PyTorch tensors into its C ABI (include/relkl.h).
 """
 from .ops import (RelationKL, make_desc, relation_kl, relkl_bwd, relkl_bwd_qkv, relkl_fwd,
-                  relkl_fwd_qkv, relkl_get_device_error, relkl_path_for, relkl_set_wait_timeout_ns,
+                  relkl_fwd_noalloc, relkl_fwd_qkv, relkl_get_device_error, relkl_path_for, relkl_set_wait_timeout_ns,
                   relkl_workspace_bytes, relkl_workspace_init, workspace)
 
 __all__ = ["RelationKL", "make_desc", "relation_kl", "relkl_bwd", "relkl_bwd_qkv", "relkl_fwd",
-           "relkl_fwd_qkv", "relkl_get_device_error", "relkl_path_for",
+           "relkl_fwd_noalloc", "relkl_fwd_qkv", "relkl_get_device_error", "relkl_path_for",
            "relkl_set_wait_timeout_ns", "relkl_workspace_bytes", "relkl_workspace_init",
            "workspace"]

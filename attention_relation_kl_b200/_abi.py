@@ -20,7 +20,7 @@ RELKL_FP32 = 1
 EXPORTS = ("relkl_workspace_bytes", "relkl_workspace_init", "relkl_fwd", "relkl_bwd",
            "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_get_device_error",
            "relkl_set_wait_timeout_ns", "relkl_status_string", "relkl_last_cuda_error",
-           "relkl_path_for")
+           "relkl_path_for", "relkl_fwd_noalloc")
 
 
 class relkl_desc(ctypes.Structure):
@@ -62,6 +62,8 @@ def _declare(lib):
     lib.relkl_last_cuda_error.argtypes = []
     lib.relkl_path_for.restype = ctypes.c_int32
     lib.relkl_path_for.argtypes = [ctypes.POINTER(relkl_desc)]
+    lib.relkl_fwd_noalloc.restype = ctypes.c_int
+    lib.relkl_fwd_noalloc.argtypes = [ctypes.POINTER(relkl_desc), _vp, _vp, _vp, _vp, _vp]
     return lib
 
 

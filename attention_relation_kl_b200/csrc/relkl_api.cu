@@ -401,3 +401,62 @@ const char* relkl_status_string(relkl_status s) {
 int32_t relkl_last_cuda_error(void) { return g_last_cuda; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// relkl_fwd_noalloc: the tensor-core forward with its scratch (the device
+// status record) in a static device array instead of a caller workspace.
+// Host code must not hand the array's name to a kernel: on the host it is a
+// stand-in, not a device address.  The address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RELKL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_addr[64];
+std::mutex g_noalloc_mu;
+
+relkl_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return RELKL_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return RELKL_OK;
+}
+}  // namespace
+
+extern "C" relkl_status relkl_fwd_noalloc(const relkl_desc* desc, const void* x_t,
+                                          const void* x_s, float* kl, float* stats,
+                                          void* stream) {
+  const void* xt[1] = {x_t};
+  const void* xs[1] = {x_s};
+  bool empty = false;
+  relkl_status s = check_multi(1, desc, xt, xs, &empty);
+  if (s != RELKL_OK || empty) return s;
+  if (!kl || !stats || !aligned(kl, 4) || !aligned(stats, 16)) return RELKL_ERR_INVALID;
+  if (!use_tc(1, desc, xt, xs)) return RELKL_ERR_UNSUPPORTED;
+  if (kWorkspaceBytes > sizeof(g_noalloc_scratch)) return RELKL_ERR_WORKSPACE;
+  DevInfo dev;
+  if ((s = device_info(&dev)) != RELKL_OK) return s;
+  if (dev.major != 10) return RELKL_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != RELKL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the record keeps the previous call's contents: clear it on this stream first
+  cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(DevStatus), st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  TcParams p;
+  if ((s = build_tc(1, desc, xt, xs, &p, scratch)) != RELKL_OK) return s;
+  float* k[1] = {kl};
+  float* sts[1] = {stats};
+  set_seg_outputs(&p, 1, desc, k, sts, nullptr, nullptr, nullptr);
+  const int grid = p.n_items < dev.sms ? p.n_items : dev.sms;
+  e = tc_launch_fwd(p, desc->d, grid, st);
+  return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
+}

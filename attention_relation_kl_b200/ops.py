@@ -21,7 +21,8 @@ from ._abi import check, relkl_desc
 
 __all__ = ["relkl_fwd", "relkl_bwd", "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_workspace_bytes",
            "relkl_workspace_init", "relkl_get_device_error", "relkl_set_wait_timeout_ns",
-           "relkl_path_for", "workspace", "make_desc", "relation_kl", "RelationKL"]
+           "relkl_path_for", "workspace", "make_desc", "relation_kl", "RelationKL",
+           "relkl_fwd_noalloc"]
 
 _DTYPES = {torch.bfloat16: _abi.RELKL_BF16, torch.float32: _abi.RELKL_FP32}
 
@@ -174,6 +175,32 @@ def relkl_bwd(x_t: torch.Tensor, x_s: torch.Tensor, stats: torch.Tensor,
     """dL/dX_s (float32) with L = sum_i dkl_i kl_i (dkl=None: 1/N per row)."""
     return relkl_bwd_qkv([(x_t, x_s)], [stats], None if dkl is None else [dkl], causal, scale,
                          out=None if dx_s is None else [dx_s], ws=ws, stream=stream)[0]
+
+
+def relkl_fwd_noalloc(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,
+                      scale: float = 0.0, *, kl: Optional[torch.Tensor] = None,
+                      stats: Optional[torch.Tensor] = None, stream=None):
+    """relkl_fwd for callers that cannot provide a device workspace.
+
+    The library call itself allocates nothing: its scratch lives in a static
+    device array inside librelkl.so.  This wrapper only allocates the outputs
+    when they are not passed in.  Tensor-core path only (bf16, d in {64, 128}).
+    Calls that overlap on the GPU share that array and race on it.
+    """
+    _cuda(x_t, "x_t")
+    _cuda(x_s, "x_s")
+    if x_t.shape != x_s.shape or x_t.stride() != x_s.stride() or x_t.dtype != x_s.dtype:
+        raise ValueError("teacher and student must share shape, strides and dtype")
+    desc = make_desc(x_t, causal, scale)
+    B, H, N, _ = x_t.shape
+    if kl is None:
+        kl = torch.empty((B, H, N), dtype=torch.float32, device=x_t.device)
+    if stats is None:
+        stats = torch.empty((B, H, N, 4), dtype=torch.float32, device=x_t.device)
+    code = _abi.lib().relkl_fwd_noalloc(ctypes.byref(desc), _ptr(x_t), _ptr(x_s), _ptr(kl),
+                                        _ptr(stats), _stream(x_t.device, stream))
+    check(code, "relkl_fwd_noalloc")
+    return kl, stats
 
 
 def relkl_get_device_error(ws: Optional[torch.Tensor] = None, stream=None) -> Tuple[int, int]:

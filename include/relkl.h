@@ -143,6 +143,33 @@ int32_t relkl_last_cuda_error(void);
  * 2 = CUDA-core float32 path, 0 = unsupported.  Validation-free.            */
 int32_t relkl_path_for(const relkl_desc* desc);
 
+/* Forward that needs no workspace from the caller and allocates nothing.
+ * The paper has no counterpart: this entry point exists for callers that
+ * cannot obtain device memory for a workspace, such as a host framework that
+ * plans every device buffer itself and hands a custom operation only its
+ * inputs and outputs.
+ *
+ * Same arguments and results as relkl_fwd, without ws / ws_bytes; tensor-core
+ * path only (bf16, d in {64, 128}; anything else returns
+ * RELKL_ERR_UNSUPPORTED).  The kernel's scratch -- the record a device-side
+ * wait writes when it runs out -- lives in a static device array of
+ * RELKL_NOALLOC_SCRATCH_BYTES bytes inside the library, which every GPU that
+ * loads the library keeps until the process exits.  A call whose scratch need
+ * (relkl_workspace_bytes()) exceeded that size would be refused with
+ * RELKL_ERR_WORKSPACE; the need does not grow with B, H or N.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and keeps it; make that first call before any
+ *    stream capture.
+ *  - All calls share the one array, which keeps what the last call wrote;
+ *    each call clears the record on its stream before its kernel starts.
+ *    Calls that overlap on the GPU (other streams, other threads) race on the
+ *    record.
+ *  - A wait that ran out is recorded but cannot be read back through this
+ *    entry point; use relkl_fwd with a workspace when that report matters.  */
+#define RELKL_NOALLOC_SCRATCH_BYTES 256
+relkl_status relkl_fwd_noalloc(const relkl_desc* desc, const void* x_t, const void* x_s,
+                               float* kl, float* stats, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
