@@ -140,6 +140,23 @@ relkl_status encode_x(CUtensorMap* m, const relkl_desc& d, const void* x) {
   return r == CUDA_SUCCESS ? RELKL_OK : RELKL_ERR_UNSUPPORTED;
 }
 
+// dX [B,H,N,d] f32 contiguous: 4-D map, box 32 cols x 32 rows, 128B swizzle,
+// the target of the backward's TMA reduce-adds.
+relkl_status encode_dx(CUtensorMap* m, const relkl_desc& d, float* dx) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return RELKL_ERR_CUDA;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.d), static_cast<cuuint64_t>(d.N),
+                              static_cast<cuuint64_t>(d.H), static_cast<cuuint64_t>(d.B)};
+  const cuuint64_t row = static_cast<cuuint64_t>(d.d) * 4;
+  const cuuint64_t strides[3] = {row, row * d.N, row * d.N * d.H};
+  const cuuint32_t box[4] = {32, 32, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dx, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RELKL_OK : RELKL_ERR_UNSUPPORTED;
+}
+
 relkl_status check_ws(const void* ws, size_t ws_bytes) {
   if (!ws || ws_bytes < kWorkspaceBytes || !aligned(ws, 256)) return RELKL_ERR_WORKSPACE;
   return RELKL_OK;
@@ -331,6 +348,10 @@ relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* c
   if (tc) {
     if ((s = build_tc(n_rel, descs, x_t, x_s, &tp, ws)) != RELKL_OK) return s;
     set_seg_outputs(&tp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);
+    for (int r = 0, seg = 0; r < n_rel; ++r) {
+      if (!n_units(descs[r])) continue;
+      if ((s = encode_dx(&tp.seg[seg++].tm_dx, descs[r], dx_s[r])) != RELKL_OK) return s;
+    }
   } else {
     build_simt(n_rel, descs, x_t, x_s, &sp);
     set_seg_outputs(&sp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);

@@ -417,19 +417,58 @@ struct BwdSmem {
   static constexpr int TILE = BM * D * 2;
   static constexpr int XT_I = 0;
   static constexpr int XS_I = TILE;
-  static constexpr int XT_R = 2 * TILE;            // teacher ring, 2 stages
-  static constexpr int XS_R = 4 * TILE;            // student ring, 2 stages
-  static constexpr int G = 6 * TILE;               // 128 x 128 bf16 gradient tile (two boxes)
-  static constexpr int BARS = G + 2 * BOX;
-  // full_I, empty_I, fullT[2], emptyT[2], fullS[2], emptyS[2], s_full, s_empty,
+  static constexpr int XT_R = 2 * TILE;            // teacher column tile, one stage
+  static constexpr int XS_R = 3 * TILE;            // student ring, two stages
+  static constexpr int G = 5 * TILE;               // 128 x 128 bf16 gradient tile (two boxes)
+  static constexpr int STG = G + 2 * BOX;          // epilogue staging: 4 warps x 2 x 4 KB
+  static constexpr int STG_BYTES = 32 * 32 * 4;    // one 32-row x 32-col f32 box
+  static constexpr int BARS = STG + 4 * 2 * STG_BYTES;
+  // full_I, empty_I, fullT, emptyT, fullS[2], emptyS[2], s_full, s_empty,
   // g_full, g_empty, p_full, p_empty, dxi_full, dxi_empty, drain
-  static constexpr int NBAR = 19;
+  static constexpr int NBAR = 17;
   static constexpr int MISC = BARS + NBAR * 8;
   static constexpr int BYTES = MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
 };
 
 constexpr int BWD_THREADS = 448;   // warps 0-7 rows, 8-11 epilogue, 12 TMA, 13 MMA
+
+// Epilogue helper: add the 32 rows x D columns a warp holds in TMEM
+// (lanes q*32.., columns col0..) into dX rows row0.. through TMA reduce-adds
+// of 32 x 32 f32 boxes staged in 128B-swizzled shared memory (two buffers per
+// warp).  Rows at or past N are skipped by TMA.
+template <int D>
+__device__ __forceinline__ void epilogue_reduce(uint32_t taddr, uint32_t stg, uint32_t& nstg,
+                                                const CUtensorMap* map, int row0, int h, int b,
+                                                int N, int lane, uint32_t release_bar) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    tmem_wait_ld();
+    if (c == D / 32 - 1) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(release_bar);
+    }
+    const uint32_t buf = stg + (nstg & 1) * (32 * 32 * 4);
+    if (lane == 0) bulk_wait_read<1>();   // this buffer's previous reduce has read it
+    __syncwarp();
+    const uint32_t rowp = buf + lane * 128;
+#pragma unroll
+    for (int k4 = 0; k4 < 8; ++k4)
+      st_shared_v4(rowp + ((k4 ^ (lane & 7)) << 4), __float_as_uint(v[4 * k4]),
+                   __float_as_uint(v[4 * k4 + 1]), __float_as_uint(v[4 * k4 + 2]),
+                   __float_as_uint(v[4 * k4 + 3]));
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (row0 < N) tma_reduce_add_4d(map, buf, c * 32, row0, h, b);
+      bulk_commit();
+    }
+    ++nstg;
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
@@ -445,14 +484,12 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
 
   const uint32_t bar0 = base + L::BARS;
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
-  const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1);
-  auto FULL_T = [&](int s) { return BAR(2 + s); };
-  auto EMPTY_T = [&](int s) { return BAR(4 + s); };
-  auto FULL_S = [&](int s) { return BAR(6 + s); };
-  auto EMPTY_S = [&](int s) { return BAR(8 + s); };
-  const uint32_t S_FULL = BAR(10), S_EMPTY = BAR(11), G_FULL = BAR(12), G_EMPTY = BAR(13);
-  const uint32_t P_FULL = BAR(14), P_EMPTY = BAR(15), DXI_FULL = BAR(16), DXI_EMPTY = BAR(17);
-  const uint32_t DRAIN = BAR(18);
+  const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1), FULL_T = BAR(2), EMPTY_T = BAR(3);
+  auto FULL_S = [&](int s) { return BAR(4 + s); };
+  auto EMPTY_S = [&](int s) { return BAR(6 + s); };
+  const uint32_t S_FULL = BAR(8), S_EMPTY = BAR(9), G_FULL = BAR(10), G_EMPTY = BAR(11);
+  const uint32_t P_FULL = BAR(12), P_EMPTY = BAR(13), DXI_FULL = BAR(14), DXI_EMPTY = BAR(15);
+  const uint32_t DRAIN = BAR(16);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
 
@@ -464,9 +501,9 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
   if (threadIdx.x == 0) {
     mbar_init(FULL_I, 1);
     mbar_init(EMPTY_I, 1);
+    mbar_init(FULL_T, 1);
+    mbar_init(EMPTY_T, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(FULL_T(s), 1);
-      mbar_init(EMPTY_T(s), 1);
       mbar_init(FULL_S(s), 1);
       mbar_init(EMPTY_S(s), 1);
     }
@@ -497,9 +534,10 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       for (int s = 0; s < p.n_seg; ++s) {
         tma_prefetch_desc(&p.seg[s].tm_t);
         tma_prefetch_desc(&p.seg[s].tm_s);
+        tma_prefetch_desc(&p.seg[s].tm_dx);
       }
-      uint32_t nI = 0, nJ = 0;
-      uint32_t armsT[2] = {0, 0}, armsS[2] = {0, 0};   // loads issued per ring stage
+      uint32_t nI = 0, nJ = 0, armsT = 0;
+      uint32_t armsS[2] = {0, 0};   // loads issued per ring stage
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
@@ -516,16 +554,17 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
           ++nI;
           const int nT = n_col_tiles(p, I);
           for (int J = 0; J < nT; ++J) {
-            const int st = nJ & 1;
-            const uint32_t par = ((nJ >> 1) & 1) ^ 1;
-            if (!(ok = mbar_wait(EMPTY_T(st), par, wc, W_TMA_EMPTY_J))) break;
-            mbar_arrive_expect_tx(FULL_T(st), L::TILE);
+            // teacher tile first: its single slot frees as soon as Z_t(J-1) is done,
+            // while a student slot frees only after the gradient MMAs of J-2
+            if (!(ok = mbar_wait(EMPTY_T, (nJ & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_T, L::TILE);
 #pragma unroll
             for (int b = 0; b < D / 64; ++b)
-              tma_load_4d(base + L::XT_R + st * L::TILE + b * BOX, &U.seg->tm_t, FULL_T(st),
-                          b * 64, J * BN, U.h, U.b);
-            ++armsT[st];
-            if (!(ok = mbar_wait(EMPTY_S(st), par, wc, W_TMA_EMPTY_J))) break;
+              tma_load_4d(base + L::XT_R + b * BOX, &U.seg->tm_t, FULL_T, b * 64, J * BN, U.h,
+                          U.b);
+            ++armsT;
+            const int st = nJ & 1;
+            if (!(ok = mbar_wait(EMPTY_S(st), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
             mbar_arrive_expect_tx(FULL_S(st), L::TILE);
 #pragma unroll
             for (int b = 0; b < D / 64; ++b)
@@ -538,10 +577,9 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       }
       // wait for the copies still in flight before the CTA may exit
       if (nI) mbar_wait_drain(FULL_I, (nI - 1) & 1, kDrainNs);
-      for (int st = 0; st < 2; ++st) {
-        if (armsT[st]) mbar_wait_drain(FULL_T(st), (armsT[st] - 1) & 1, kDrainNs);
+      if (armsT) mbar_wait_drain(FULL_T, (armsT - 1) & 1, kDrainNs);
+      for (int st = 0; st < 2; ++st)
         if (armsS[st]) mbar_wait_drain(FULL_S(st), (armsS[st] - 1) & 1, kDrainNs);
-      }
     }
     __syncwarp();
   } else if (warp == 13) {
@@ -590,15 +628,15 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
           int prev_st = -1;
           for (int J = 0; J < nT; ++J) {
             const int st = nJ & 1;
-            const uint32_t par = (nJ >> 1) & 1;
-            if (!(ok = mbar_wait(FULL_T(st), par, wc, W_MMA_FULL_J))) break;
-            if (!(ok = mbar_wait(FULL_S(st), par, wc, W_MMA_FULL_J))) break;
+            if (!(ok = mbar_wait(FULL_T, nJ & 1, wc, W_MMA_FULL_J))) break;
             if (!(ok = mbar_wait(S_EMPTY, (ns & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
             tc_fence_after();
-            issue_logits<D>(tmem + T_ST, base + L::XT_I, base + L::XT_R + st * L::TILE);
-            issue_logits<D>(tmem + T_SS, base + L::XS_I, base + L::XS_R + st * L::TILE);
+            issue_logits<D>(tmem + T_ST, base + L::XT_I, base + L::XT_R);
             issued = true;
-            umma_commit(EMPTY_T(st));
+            umma_commit(EMPTY_T);   // the teacher tile is free as soon as Z_t is done
+            if (!(ok = mbar_wait(FULL_S(st), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+            tc_fence_after();
+            issue_logits<D>(tmem + T_SS, base + L::XS_I, base + L::XS_R + st * L::TILE);
             umma_commit(S_FULL);
             ++ns;
             ++nJ;
@@ -622,40 +660,23 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
   } else if (warp >= 8) {
     // ------------------------------------------------------- epilogue
     const int q = warp - 8;
-    uint32_t np = 0, nrb = 0;
+    const uint32_t stg = base + L::STG + q * 2 * L::STG_BYTES;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t np = 0, nrb = 0, nstg = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
       const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
       const Unit U = decode_unit(p, u);
-      float* dx = U.seg->dx + U.row0 * D;
       for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
         const int I = pass_block(p, pp, pass);
         const int nT = n_col_tiles(p, I);
-        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
         for (int J = 0; J < nT; ++J) {
           ok = mbar_wait(P_FULL, np & 1, wc, W_EPI_P_FULL);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
-          const int jrow = J * BN + q * 32 + lane;
-          float* dst = dx + static_cast<long long>(jrow) * D;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float v[32];
-            tmem_ld32(tmem + lane_addr + T_P + c * 32, v);
-            tmem_wait_ld();
-            if (c == D / 32 - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(P_EMPTY);
-            }
-            if (jrow < p.N) {
-#pragma unroll
-              for (int k = 0; k < 8; ++k)
-                red_add_v4(dst + c * 32 + 4 * k, v[4 * k], v[4 * k + 1], v[4 * k + 2],
-                           v[4 * k + 3]);
-            }
-          }
+          epilogue_reduce<D>(tmem + lane_addr + T_P, stg, nstg, &U.seg->tm_dx, J * BN + q * 32,
+                             U.h, U.b, p.N, lane, P_EMPTY);
           ++np;
         }
         if (!ok) break;
@@ -663,27 +684,13 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const int irow = I * BM + q * 32 + lane;
-        float* dst = dx + static_cast<long long>(irow) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tmem_ld32(tmem + lane_addr + T_DXI + c * 32, v);
-          tmem_wait_ld();
-          if (c == D / 32 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(DXI_EMPTY);
-          }
-          if (irow < p.N) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              red_add_v4(dst + c * 32 + 4 * k, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-          }
-        }
+        epilogue_reduce<D>(tmem + lane_addr + T_DXI, stg, nstg, &U.seg->tm_dx, I * BM + q * 32,
+                           U.h, U.b, p.N, lane, DXI_EMPTY);
         ++nrb;
       }
     }
+    if (lane == 0) bulk_wait_all();   // reduces must finish reading staging before exit
+    __syncwarp();
   } else {
     // --------------------------------------------------- row warpgroups
     const int q = warp & 3;
