@@ -120,7 +120,7 @@ float logit_scale(const relkl_desc& d) {
   return d.scale > 0.f ? d.scale : 1.0f / std::sqrt(static_cast<float>(d.d));
 }
 
-relkl_status encode_x(CUtensorMap* m, const relkl_desc& d, const void* x) {
+relkl_status encode_x(CUtensorMap* m, const relkl_desc& d, const void* x, cuuint32_t box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return RELKL_ERR_CUDA;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.d), static_cast<cuuint64_t>(d.N),
@@ -132,7 +132,7 @@ relkl_status encode_x(CUtensorMap* m, const relkl_desc& d, const void* x) {
   const int64_t row = d.stride[2] > 0 ? d.stride[2] : d.d;
   const cuuint64_t strides[3] = {stride_or(2, d.d), stride_or(1, row * d.N),
                                  stride_or(0, row * d.N * d.H)};
-  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t box[4] = {64, box_rows, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -350,7 +350,11 @@ relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* c
     set_seg_outputs(&tp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);
     for (int r = 0, seg = 0; r < n_rel; ++r) {
       if (!n_units(descs[r])) continue;
-      if ((s = encode_dx(&tp.seg[seg++].tm_dx, descs[r], dx_s[r])) != RELKL_OK) return s;
+      TcSeg& sg = tp.seg[seg++];
+      if ((s = encode_dx(&sg.tm_dx, descs[r], dx_s[r])) != RELKL_OK) return s;
+      // 64-row boxes for the column tiles of the d = 128 backward
+      if ((s = encode_x(&sg.tm_t64, descs[r], x_t[r], 64)) != RELKL_OK) return s;
+      if ((s = encode_x(&sg.tm_s64, descs[r], x_s[r], 64)) != RELKL_OK) return s;
     }
   } else {
     build_simt(n_rel, descs, x_t, x_s, &sp);

@@ -104,6 +104,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// mbar_wait for a converged warp: every lane waits and the warp agrees on the
+// outcome, so the loop around it never diverges.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtl& c,
+                                               unsigned int where) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, c, where));
+}
+
 // Unconditional bounded wait used only on the way out (in-flight copies).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
                                                 unsigned long long limit_ns) {
@@ -219,6 +226,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
       : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 // ------------------------------------------------------- UMMA descriptors
 // Shared-memory matrix descriptor (tcgen05 format, version 1) for the
 // 128-byte swizzle: start address, leading- and stride-dimension byte
@@ -235,6 +255,68 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for tcgen05
   d |= static_cast<uint64_t>(2) << 61;  // 128-byte swizzle
   return d;
+}
+
+// The same descriptor split into its two 32-bit words, so that the issuing
+// thread can precompute one word pair per shared-memory buffer and step along
+// K by adding an immediate (start address >> 4) to the low word; addresses
+// below 256 KB never carry out of the 14-bit field.
+__host__ __device__ constexpr uint32_t sw128_desc_lo(uint32_t saddr, uint32_t lbo) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sw128_desc_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+
+// D[tmem] (+)= A * B with descriptors passed as word pairs.
+__device__ __forceinline__ void umma_bf16_w(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                            uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Variants for a converged warp: every lane runs the issuing loop (so the
+// descriptor words stay warp-uniform) and only the lane whose `leader` is
+// non-zero issues the instruction.
+__device__ __forceinline__ uint32_t elect_leader() {
+  uint32_t is_leader;
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, e;\n\t}"
+      : "=r"(is_leader));
+  return is_leader;
+}
+
+__device__ __forceinline__ void umma_bf16_w_lead(uint32_t leader, uint32_t d_tmem, uint32_t a_lo,
+                                                 uint32_t a_hi, uint32_t b_lo, uint32_t b_hi,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 e, %7, 0;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\t"
+      "mov.b64 db, {%3, %4};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate), "r"(leader)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_lead(uint32_t leader, uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "setp.ne.b32 e, %1, 0;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar),
+      "r"(leader)
+      : "memory");
 }
 
 // Instruction descriptor, kind::f16: bf16 x bf16 -> f32, dense.
@@ -256,9 +338,61 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x for a pair of arguments on the FMA pipe instead of MUFU, for x <= 0
+// (arguments below -125 are clamped; their results are < 2^-125).
+// Cody and Waite's reduction x = n + f with n = rint(x), f in [-1/2, 1/2]
+// (n comes from adding 1.5 * 2^23, which leaves rint(x) in the low mantissa
+// bits), a polynomial p(f) ~ 2^f with minimax relative error fitted by
+// csrc/fit_exp2_poly.py, and n added to p's exponent field with one integer
+// multiply-add.  DEG 5: relative error 1.8e-7 (float32 evaluation, on par with
+// ex2.approx); DEG 3: 1.0e-4.
+template <int DEG>
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  static_assert(DEG == 3 || DEG == 5, "fitted degrees are 3 and 5");
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
+  float2 p;
+  if constexpr (DEG == 5) {
+    p = __ffma2_rn(make_float2(1.326627913e-03f, 1.326627913e-03f), f,
+                   make_float2(9.671512060e-03f, 9.671512060e-03f));
+    p = __ffma2_rn(p, f, make_float2(5.550728366e-02f, 5.550728366e-02f));
+    p = __ffma2_rn(p, f, make_float2(2.402224243e-01f, 2.402224243e-01f));
+    p = __ffma2_rn(p, f, make_float2(6.931470037e-01f, 6.931470037e-01f));
+  } else {
+    p = __ffma2_rn(make_float2(5.502312258e-02f, 5.502312258e-02f), f,
+                   make_float2(2.422109395e-01f, 2.422109395e-01f));
+    p = __ffma2_rn(p, f, make_float2(6.932800412e-01f, 6.932800412e-01f));
+  }
+  p = __ffma2_rn(p, f, make_float2(1.0f, 1.0f));
+  // the low 9 bits of t's pattern hold n (two's complement); shifted by 23
+  // they land on the exponent field (unsigned arithmetic wraps mod 2^32)
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+__device__ __forceinline__ float2 ex2_approx2(float2 x) {
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// The same packing with integer instructions only: round to nearest even
+// (add 0x7FFF plus the lowest kept bit, keep the high half), then take the two
+// high halves with one byte permute.  Inputs are finite.
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
+  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+  a += 0x7FFFu + ((a >> 16) & 1u);
+  b += 0x7FFFu + ((b >> 16) & 1u);
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 
@@ -267,6 +401,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
+}
+
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, float v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(__float_as_uint(v)) : "memory");
 }
 
 __device__ __forceinline__ void red_add_v4(float* gaddr, float a, float b, float c, float d) {

@@ -16,6 +16,8 @@ struct TcSeg {
   CUtensorMap tm_t;          // teacher [B,H,N,d] bf16, box 64 cols x 128 rows, 128B swizzle
   CUtensorMap tm_s;          // student, same geometry
   CUtensorMap tm_dx;         // dX [B,H,N,d] f32, box 32 cols x 32 rows, 128B swizzle (bwd)
+  CUtensorMap tm_t64;        // teacher, box 64 cols x 64 rows (bwd column tiles, d = 128)
+  CUtensorMap tm_s64;        // student, same geometry
   float* kl;                 // [B,H,N]
   float* stats;              // [B,H,N,4]
   const float* dkl;          // [B,H,N] or null (1/N)

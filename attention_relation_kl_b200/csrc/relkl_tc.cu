@@ -45,6 +45,25 @@ constexpr int BM = 128;        // rows of a row block (TMEM lanes)
 constexpr int BN = 128;        // columns of a logit tile
 constexpr int BOX = 128 * 128;  // bytes of one 128-row x 64-col bf16 box
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Which column pairs take 2^x on the FMA pipe (exp2_poly2) instead of MUFU.
+// Measured on B200: MUFU ex2 costs 8 clk per warp instruction (4 lanes/clk per
+// SMSP); the degree-3 packed polynomial costs ~19.5 clk per pair of exps on
+// the FMA pipe (FFMA2 is 2 clk, not 1), and the FMA pipe already carries the
+// exp arguments, differences and accumulations of every entry.  In both
+// kernels moving exps off MUFU therefore lengthened the exp pass, so no pair
+// is offloaded unless RELKL_EXP2_POLY is defined (forward: 4 of 16 pairs with
+// the degree-5 fit; backward: 3 of 8 pairs with the degree-3 fit).
+#ifdef RELKL_EXP2_POLY
+__host__ __device__ constexpr bool fwd_poly_pair(int pair) { return (pair & 3) == 3; }
+__host__ __device__ constexpr bool bwd_poly_pair(int pair) {
+  return (pair & 7) == 2 || (pair & 7) == 5 || (pair & 7) == 7;
+}
+#else
+__host__ __device__ constexpr bool fwd_poly_pair(int) { return false; }
+__host__ __device__ constexpr bool bwd_poly_pair(int) { return false; }
+#endif
+
 constexpr unsigned long long kDrainNs = 200000000ull;  // 0.2 s for in-flight copies
 
 struct Unit {
@@ -93,6 +112,20 @@ __device__ __forceinline__ void issue_logits(uint32_t acc, uint32_t a_base, uint
   }
 }
 
+// Same K-loop with precomputed descriptor words: a_lo and b_lo name the first
+// 64-column box of 128-row tiles (boxes 16 KB apart), steps of 32 B in a row.
+template <int D>
+__device__ __forceinline__ void issue_logits_w(uint32_t lead, uint32_t acc, uint32_t a_lo,
+                                               uint32_t b_lo) {
+  constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+  constexpr uint32_t hi = sw128_desc_hi(1024);
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint32_t off = (k >> 2) * (BOX >> 4) + (k & 3) * 2;
+    umma_bf16_w_lead(lead, acc, a_lo + off, hi, b_lo + off, hi, idesc, k > 0 ? 1u : 0u);
+  }
+}
+
 // =========================================================================
 //                                FORWARD
 // =========================================================================
@@ -103,8 +136,8 @@ struct FwdSmem {
   static constexpr int XS_I = TILE;
   static constexpr int RING = 2 * TILE;              // stage k: xt at RING + 2k*TILE, xs after it
   static constexpr int STAGES = 2;
-  static constexpr int MERGE = RING + STAGES * 2 * TILE;  // float4 per row
-  static constexpr int BARS = MERGE + BM * 16;
+  static constexpr int MERGE = RING + STAGES * 2 * TILE;  // float4 per row, 3 column quarters
+  static constexpr int BARS = MERGE + 3 * BM * 16;
   // barriers: full_I, empty_I, full_J[2], empty_J[2], tf[2], te[2], mfull, mempty, drain
   static constexpr int NBAR = 13;
   static constexpr int MISC = BARS + NBAR * 8;       // tmem base (u32) + abort flag (int)
@@ -112,7 +145,10 @@ struct FwdSmem {
   static constexpr int ALLOC = BYTES + 1024;         // slack for 1024-byte alignment
 };
 
-constexpr int FWD_THREADS = 320;   // warps 0-7 rows, 8 TMA, 9 MMA
+// Warps 0-15: four row warpgroups, warpgroup k owning columns [32k, 32k+32)
+// of every tile; warp 16 TMA; warp 17 MMA.
+constexpr int FWD_THREADS = 576;
+constexpr int FWD_TMA_WARP = 16, FWD_MMA_WARP = 17;
 
 template <int D>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
@@ -147,15 +183,15 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
       mbar_init(FULL_J(s), 1);
       mbar_init(EMPTY_J(s), 1);
       mbar_init(TF(s), 1);
-      mbar_init(TE(s), 8);
+      mbar_init(TE(s), 16);
     }
-    mbar_init(MFULL, 4);
+    mbar_init(MFULL, 12);
     mbar_init(MEMPTY, 4);
     mbar_init(DRAIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == FWD_MMA_WARP) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -164,7 +200,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == FWD_TMA_WARP) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
       for (int s = 0; s < p.n_seg; ++s) {
@@ -210,41 +246,47 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == FWD_MMA_WARP) {
     // ------------------------------------------------------------ MMA
-    if (lane == 0) {
+    // The whole warp runs this loop (descriptor words stay warp-uniform); one
+    // elected lane issues the MMAs and commits.
+    {
+      const uint32_t lead = elect_leader();
       uint32_t nI = 0, nJ = 0, nt = 0;
       bool ok = true, issued = false;
+      const uint32_t dXtI = sw128_desc_lo(base + L::XT_I, 16);
+      const uint32_t dXsI = sw128_desc_lo(base + L::XS_I, 16);
+      const uint32_t ring0 = sw128_desc_lo(base + L::RING, 16);
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
         (void)u;
         for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
           const int I = pass_block(p, pp, pass);
-          if (!(ok = mbar_wait(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
+          if (!(ok = mbar_wait_warp(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
           const int nT = n_col_tiles(p, I);
           for (int J = 0; J < nT; ++J) {
             const int st = nJ & 1;
             const int buf = nt & 1;
-            if (!(ok = mbar_wait(FULL_J(st), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
-            if (!(ok = mbar_wait(TE(buf), ((nt >> 1) & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
+            if (!(ok = mbar_wait_warp(FULL_J(st), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+            if (!(ok = mbar_wait_warp(TE(buf), ((nt >> 1) & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
             tc_fence_after();
-            const uint32_t xt = base + L::RING + st * 2 * L::TILE;
+            const uint32_t xt = ring0 + st * (2 * L::TILE >> 4);
             const uint32_t acc = tmem + buf * 256;
-            issue_logits<D>(acc, base + L::XT_I, xt);
-            issue_logits<D>(acc + 128, base + L::XS_I, xt + L::TILE);
+            issue_logits_w<D>(lead, acc, dXtI, xt);
+            issue_logits_w<D>(lead, acc + 128, dXsI, xt + (L::TILE >> 4));
             issued = true;
-            umma_commit(EMPTY_J(st));
-            umma_commit(TF(buf));
+            umma_commit_lead(lead, EMPTY_J(st));
+            umma_commit_lead(lead, TF(buf));
             ++nJ;
             ++nt;
           }
           if (!ok) break;
-          umma_commit(EMPTY_I);
+          umma_commit_lead(lead, EMPTY_I);
           ++nI;
         }
       }
       if (issued) {
-        umma_commit(DRAIN);
+        umma_commit_lead(lead, DRAIN);
         mbar_wait_drain(DRAIN, 0, kDrainNs);
       }
     }
@@ -252,7 +294,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
   } else {
     // --------------------------------------------------- row warpgroups
     const int q = warp & 3;      // TMEM lane quarter
-    const int half = warp >> 2;  // column half of each tile
+    const int wg = warp >> 2;    // column quarter of each tile
     const int r = q * 32 + lane;
     const float sl2 = p.sl2;
     uint32_t nt = 0, nm = 0;
@@ -265,126 +307,144 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
         const int row = I * BM + r;
         const int nT = n_col_tiles(p, I);
         float m_run = -INFINITY;
-        float S[4] = {0.f, 0.f, 0.f, 0.f}, C[4] = {0.f, 0.f, 0.f, 0.f},
-              A[4] = {0.f, 0.f, 0.f, 0.f};
+        // running sums, two float2 lanes each: S_t, C = sum(e_s - e_t), A = sum e_t (z_t - z_s)
+        float2 S2[2], C2[2], A2[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) S2[k] = C2[k] = A2[k] = make_float2(0.f, 0.f);
         for (int J = 0; J < nT; ++J) {
           const int buf = nt & 1;
           ok = mbar_wait(TF(buf), (nt >> 1) & 1, wc, W_SM_S_FULL);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + half * 64;
-          float t0[32], s0[32], t1[32], s1[32];
-          tmem_ld32(ta, t0);
-          tmem_ld32(ta + 128, s0);
-          tmem_ld32(ta + 32, t1);
-          tmem_ld32(ta + 160, s1);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(TE(buf));
-          ++nt;
-
-          const int col0 = J * BN + half * 64;
-          const bool need_mask = (p.causal && J == I) || (col0 + 64 > p.N);
-          if (!need_mask) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int k = 0; k < 32; ++k)
-              mx = fmaxf(mx, fmaxf(fmaxf(t0[k], s0[k]), fmaxf(t1[k], s1[k])));
-            if (mx > m_run) {
-              const float a = ex2_approx((m_run - mx) * sl2);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                S[k] *= a;
-                C[k] *= a;
-                A[k] *= a;
-              }
-              m_run = mx;
+          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + wg * 32;
+          // two 16-column halves: fewer live registers, more exps in flight.  The
+          // TMEM buffer is handed back after the second load (the MMA warp only
+          // needs it again two tiles later).
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            float t[16], s[16];
+            tmem_ld16(ta + hh * 16, t);
+            tmem_ld16(ta + 128 + hh * 16, s);
+            tmem_wait_ld();
+            if (hh == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(TE(buf));
             }
-            const float nb = -m_run * sl2;
+            const int col0 = J * BN + wg * 32 + hh * 16;
+            const bool need_mask = (p.causal && J == I) || (col0 + 16 > p.N);
+            if (!need_mask) {
+              float m4[4];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const float et = ex2_approx(fmaf(t0[k], sl2, nb));
-              const float es = ex2_approx(fmaf(s0[k], sl2, nb));
-              S[k & 3] += et;
-              C[k & 3] += es - et;
-              A[k & 3] = fmaf(et, t0[k] - s0[k], A[k & 3]);
-            }
+              for (int k = 0; k < 4; ++k) m4[k] = fmaxf(t[k], s[k]);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const float et = ex2_approx(fmaf(t1[k], sl2, nb));
-              const float es = ex2_approx(fmaf(s1[k], sl2, nb));
-              S[k & 3] += et;
-              C[k & 3] += es - et;
-              A[k & 3] = fmaf(et, t1[k] - s1[k], A[k & 3]);
-            }
-          } else {
-            // diagonal or ragged tile: per-entry predicate
-            const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;  // last allowed column
-            float mx = -INFINITY;
+              for (int k = 4; k < 16; ++k) m4[k & 3] = fmaxf(m4[k & 3], fmaxf(t[k], s[k]));
+              const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+              if (mx > m_run) {
+                const float a = ex2_approx((m_run - mx) * sl2);
+                const float2 a2 = make_float2(a, a);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              if (col0 + k <= lim) mx = fmaxf(mx, fmaxf(t0[k], s0[k]));
-              if (col0 + 32 + k <= lim) mx = fmaxf(mx, fmaxf(t1[k], s1[k]));
-            }
-            if (mx > m_run) {
-              const float a = ex2_approx((m_run - mx) * sl2);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                S[k] *= a;
-                C[k] *= a;
-                A[k] *= a;
-              }
-              m_run = mx;
-            }
-            if (m_run > -INFINITY) {
-              const float nb = -m_run * sl2;
-#pragma unroll
-              for (int k = 0; k < 32; ++k) {
-                if (col0 + k <= lim) {
-                  const float et = ex2_approx(fmaf(t0[k], sl2, nb));
-                  const float es = ex2_approx(fmaf(s0[k], sl2, nb));
-                  S[k & 3] += et;
-                  C[k & 3] += es - et;
-                  A[k & 3] = fmaf(et, t0[k] - s0[k], A[k & 3]);
+                for (int k = 0; k < 2; ++k) {
+                  S2[k] = __fmul2_rn(S2[k], a2);
+                  C2[k] = __fmul2_rn(C2[k], a2);
+                  A2[k] = __fmul2_rn(A2[k], a2);
                 }
-                if (col0 + 32 + k <= lim) {
-                  const float et = ex2_approx(fmaf(t1[k], sl2, nb));
-                  const float es = ex2_approx(fmaf(s1[k], sl2, nb));
-                  S[k & 3] += et;
-                  C[k & 3] += es - et;
-                  A[k & 3] = fmaf(et, t1[k] - s1[k], A[k & 3]);
+                m_run = mx;
+              }
+              const float nb = -m_run * sl2;
+              const float2 sl2v = make_float2(sl2, sl2), nbv = make_float2(nb, nb);
+              const float2 m1 = make_float2(-1.f, -1.f);
+#pragma unroll
+              for (int k = 0; k < 16; k += 2) {
+                const float2 tv = make_float2(t[k], t[k + 1]);
+                const float2 sv = make_float2(s[k], s[k + 1]);
+                const float2 at = __ffma2_rn(tv, sl2v, nbv);
+                const float2 as = __ffma2_rn(sv, sl2v, nbv);
+                float2 et, es;
+                if (fwd_poly_pair(k >> 1)) {
+                  et = exp2_poly2<5>(at);
+                  es = exp2_poly2<5>(as);
+                } else {
+                  et = ex2_approx2(at);
+                  es = ex2_approx2(as);
+                }
+                const int a = (k >> 1) & 1;
+                S2[a] = __fadd2_rn(S2[a], et);
+                C2[a] = __fadd2_rn(C2[a], __ffma2_rn(et, m1, es));
+                A2[a] = __ffma2_rn(et, __ffma2_rn(sv, m1, tv), A2[a]);
+              }
+            } else {
+              // diagonal or ragged tile: per-entry predicate
+              const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;  // last allowed column
+              float mx = -INFINITY;
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+                if (col0 + k <= lim) mx = fmaxf(mx, fmaxf(t[k], s[k]));
+              if (mx > m_run) {
+                const float a = ex2_approx((m_run - mx) * sl2);
+                const float2 a2 = make_float2(a, a);
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                  S2[k] = __fmul2_rn(S2[k], a2);
+                  C2[k] = __fmul2_rn(C2[k], a2);
+                  A2[k] = __fmul2_rn(A2[k], a2);
+                }
+                m_run = mx;
+              }
+              if (m_run > -INFINITY) {
+                const float nb = -m_run * sl2;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                  if (col0 + k <= lim) {
+                    const float et = ex2_approx(fmaf(t[k], sl2, nb));
+                    const float es = ex2_approx(fmaf(s[k], sl2, nb));
+                    float2& Sa = S2[(k >> 1) & 1];
+                    float2& Ca = C2[(k >> 1) & 1];
+                    float2& Aa = A2[(k >> 1) & 1];
+                    if (k & 1) {
+                      Sa.y += et;
+                      Ca.y += es - et;
+                      Aa.y = fmaf(et, t[k] - s[k], Aa.y);
+                    } else {
+                      Sa.x += et;
+                      Ca.x += es - et;
+                      Aa.x = fmaf(et, t[k] - s[k], Aa.x);
+                    }
+                  }
                 }
               }
             }
           }
+          ++nt;
         }
         if (!ok) break;
-        const float Sx = (S[0] + S[1]) + (S[2] + S[3]);
-        const float Cx = (C[0] + C[1]) + (C[2] + C[3]);
-        const float Ax = (A[0] + A[1]) + (A[2] + A[3]);
-        // merge the two column halves through shared memory
-        if (half == 1) {
+        const float Sx = (S2[0].x + S2[0].y) + (S2[1].x + S2[1].y);
+        const float Cx = (C2[0].x + C2[0].y) + (C2[1].x + C2[1].y);
+        const float Ax = (A2[0].x + A2[0].y) + (A2[1].x + A2[1].y);
+        // merge the four column quarters through shared memory
+        if (wg != 0) {
           ok = mbar_wait(MEMPTY, (nm & 1) ^ 1, wc, W_SM_S_FULL);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          merge[r] = make_float4(m_run, Sx, Cx, Ax);
+          merge[(wg - 1) * BM + r] = make_float4(m_run, Sx, Cx, Ax);
           __syncwarp();
           if (lane == 0) mbar_arrive(MFULL);
         } else {
           ok = mbar_wait(MFULL, nm & 1, wc, W_SM_S_FULL);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          const float4 o = merge[r];
+          const float4 o1 = merge[r], o2 = merge[BM + r], o3 = merge[2 * BM + r];
           __syncwarp();
           if (lane == 0) mbar_arrive(MEMPTY);
-          const float M = fmaxf(m_run, o.x);
+          const float M = fmaxf(fmaxf(m_run, o1.x), fmaxf(o2.x, o3.x));
           const float a0 = ex2_approx((m_run - M) * sl2);
-          const float a1 = ex2_approx((o.x - M) * sl2);
-          const float St = Sx * a0 + o.y * a1;
-          const float Ct = Cx * a0 + o.z * a1;
-          const float At = Ax * a0 + o.w * a1;
+          const float a1 = ex2_approx((o1.x - M) * sl2);
+          const float a2 = ex2_approx((o2.x - M) * sl2);
+          const float a3 = ex2_approx((o3.x - M) * sl2);
+          const float St = (Sx * a0 + o1.y * a1) + (o2.y * a2 + o3.y * a3);
+          const float Ct = (Cx * a0 + o1.z * a1) + (o2.z * a2 + o3.z * a3);
+          const float At = (Ax * a0 + o1.w * a1) + (o2.w * a2 + o3.w * a3);
           if (row < p.N) {
             const float mz = M * p.scale;
             const float lse_t = mz + logf(St);
@@ -403,7 +463,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == FWD_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -431,7 +491,10 @@ struct BwdSmem {
   static constexpr int ALLOC = BYTES + 1024;
 };
 
-constexpr int BWD_THREADS = 448;   // warps 0-7 rows, 8-11 epilogue, 12 TMA, 13 MMA
+// Warps 0-15: four row warpgroups (columns [32k, 32k+32) of every tile);
+// warps 16-19: epilogue; warp 20: TMA; warp 21: MMA.
+constexpr int BWD_THREADS = 704;
+constexpr int BWD_EPI_WARP = 16, BWD_TMA_WARP = 20, BWD_MMA_WARP = 21;
 
 // Epilogue helper: add the 32 rows x D columns a warp holds in TMEM
 // (lanes q*32.., columns col0..) into dX rows row0.. through TMA reduce-adds
@@ -508,8 +571,8 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       mbar_init(EMPTY_S(s), 1);
     }
     mbar_init(S_FULL, 1);
-    mbar_init(S_EMPTY, 8);
-    mbar_init(G_FULL, 8);
+    mbar_init(S_EMPTY, 16);
+    mbar_init(G_FULL, 16);
     mbar_init(G_EMPTY, 1);
     mbar_init(P_FULL, 1);
     mbar_init(P_EMPTY, 4);
@@ -519,7 +582,7 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 13) {
+  if (warp == BWD_MMA_WARP) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -528,7 +591,7 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 12) {
+  if (warp == BWD_TMA_WARP) {
     // ------------------------------------------------------------ TMA
     if (lane == 0) {
       for (int s = 0; s < p.n_seg; ++s) {
@@ -582,7 +645,7 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
         if (armsS[st]) mbar_wait_drain(FULL_S(st), (armsS[st] - 1) & 1, kDrainNs);
     }
     __syncwarp();
-  } else if (warp == 13) {
+  } else if (warp == BWD_MMA_WARP) {
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t IDESC_GX = idesc_bf16_f32(BM, D, 0, 1);   // A = G (K-major), B = X (MN)
@@ -657,9 +720,9 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       }
     }
     __syncwarp();
-  } else if (warp >= 8) {
+  } else if (warp >= BWD_EPI_WARP) {
     // ------------------------------------------------------- epilogue
-    const int q = warp - 8;
+    const int q = warp - BWD_EPI_WARP;
     const uint32_t stg = base + L::STG + q * 2 * L::STG_BYTES;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     uint32_t np = 0, nrb = 0, nstg = 0;
@@ -694,10 +757,11 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
   } else {
     // --------------------------------------------------- row warpgroups
     const int q = warp & 3;
-    const int half = warp >> 2;
+    const int wg = warp >> 2;      // column quarter of each tile
     const int r = q * 32 + lane;
     const float sl2 = p.sl2;
-    const uint32_t gsm = base + L::G + half * BOX + r * 128;
+    // this thread's 64-byte slice of row r of the G tile: box wg/2, chunks 4*(wg&1)..+3
+    const uint32_t gsm = base + L::G + (wg >> 1) * BOX + r * 128;
     uint32_t ns = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -722,46 +786,50 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + half * 64;
-          const int col0 = J * BN + half * 64;
-          const bool need_mask = !rvalid || (col0 + 63 > lim);
+          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + wg * 32;
+          float t[32], s[32];
+          tmem_ld32(ta + T_ST, t);
+          tmem_ld32(ta + T_SS, s);
+          tmem_wait_ld();
+          // hand the logit tiles back at once: the next tile's MMAs overlap this one
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(S_EMPTY);
+          const int col0 = J * BN + wg * 32;
+          const bool need_mask = !rvalid || (col0 + 31 > lim);
+          uint32_t pk[16];
+          const float2 sl2v = make_float2(sl2, sl2), btv = make_float2(bt, bt),
+                       bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
+                       m1 = make_float2(-1.f, -1.f);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float t[32], s[32];
-            tmem_ld32(ta + T_ST + c * 32, t);
-            tmem_ld32(ta + T_SS + c * 32, s);
-            tmem_wait_ld();
-            if (c == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(S_EMPTY);
+          for (int k = 0; k < 32; k += 2) {
+            const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
+            const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
+            float2 et, es;
+            if (bwd_poly_pair(k >> 1)) {
+              et = exp2_poly2<3>(at);
+              es = exp2_poly2<3>(as);
+            } else {
+              et = ex2_approx2(at);
+              es = ex2_approx2(as);
             }
-            uint32_t pk[16];
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              float g0 = mul * (ex2_approx(fmaf(s[k], sl2, bs)) - ex2_approx(fmaf(t[k], sl2, bt)));
-              float g1 = mul * (ex2_approx(fmaf(s[k + 1], sl2, bs)) -
-                                ex2_approx(fmaf(t[k + 1], sl2, bt)));
-              if (need_mask) {
-                g0 = (col0 + c * 32 + k <= lim) ? g0 : 0.f;
-                g1 = (col0 + c * 32 + k + 1 <= lim) ? g1 : 0.f;
-              }
-              pk[k >> 1] = pack_bf16x2(g0, g1);
+            float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
+            if (need_mask) {
+              g.x = (col0 + k <= lim) ? g.x : 0.f;
+              g.y = (col0 + k + 1 <= lim) ? g.y : 0.f;
             }
-            if (c == 0) {
-              // the G buffer is free once the previous tile's gradient MMAs completed
-              ok = mbar_wait(G_EMPTY, (ns & 1) ^ 1, wc, W_SM_G_EMPTY);
-              ok = __all_sync(0xffffffffu, ok);
-              if (!ok) break;
-            }
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const int cc = c * 4 + q4;  // 16-byte chunk within the 128-byte row
-              st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[4 * q4], pk[4 * q4 + 1],
-                           pk[4 * q4 + 2], pk[4 * q4 + 3]);
-            }
+            pk[k >> 1] = pack_bf16x2(g.x, g.y);
           }
+          // the G buffer is free once the previous tile's gradient MMAs completed
+          ok = mbar_wait(G_EMPTY, (ns & 1) ^ 1, wc, W_SM_G_EMPTY);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int cc = (wg & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
+            st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2],
+                         pk[4 * q4 + 3]);
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(G_FULL);
@@ -773,7 +841,424 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == BWD_MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// =========================================================================
+//              BACKWARD, d = 128: 64-column tiles, double-buffered
+// =========================================================================
+// Same mathematics as relkl_bwd_tc_kernel with column tiles of 64: the logit
+// tiles (2 x 64 TMEM columns), the gradient tile G (16 KB) and the transposed
+// column-side product P^T = X_s[I]^T G (64 TMEM columns, M = d = 128) are all
+// double-buffered, and the student column tiles pass through a 4-stage ring, so
+// that the exp pass of tile t overlaps the logit MMAs of tile t+1 and the
+// gradient MMAs of tile t-1 without waiting on a shared buffer.
+//   TMEM: Z_t/Z_s buffers 0..255 (128 per buffer), dX_I 256..383, P^T 384..511.
+//   smem: X_t[I], X_s[I] 32 KB each; teacher ring 2 x 16 KB; student ring
+//         4 x 16 KB; G 2 x 16 KB; epilogue staging 32 KB.
+struct Bwd64Smem {
+  static constexpr int TILE_I = BM * 128 * 2;        // 128 rows: boxes of 128 x 64 (16 KB)
+  static constexpr int TILE_J = 64 * 128 * 2;        // 64 rows: boxes of 64 x 64 (8 KB)
+  static constexpr int BOX_J = 64 * 128;
+  static constexpr int XT_I = 0;
+  static constexpr int XS_I = TILE_I;
+  static constexpr int XT_R = 2 * TILE_I;            // 2 stages
+  static constexpr int XS_R = XT_R + 2 * TILE_J;     // 4 stages
+  static constexpr int G = XS_R + 4 * TILE_J;        // 2 x (128 x 64 bf16)
+  static constexpr int G_BYTES = BM * 64 * 2;
+  static constexpr int STG = G + 2 * G_BYTES;
+  static constexpr int STG_BYTES = 32 * 32 * 4;
+  static constexpr int BARS = STG + 4 * 2 * STG_BYTES;
+  // full_I, empty_I, fullT[2], emptyT[2], fullS[4], emptyS[4], s_full[2], s_empty[2],
+  // g_full[2], g_empty[2], p_full[2], p_empty[2], dxi_full, dxi_empty, drain
+  static constexpr int NBAR = 31;
+  static constexpr int MISC = BARS + NBAR * 8;
+  static constexpr int BYTES = MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+};
+static_assert(Bwd64Smem::ALLOC <= 232448, "backward shared memory exceeds 227 KB");
+
+constexpr int BN64 = 64;
+
+__device__ __forceinline__ int n_col_tiles64(const TcParams& p, int I) {
+  const int nb64 = (p.N + BN64 - 1) / BN64;
+  return p.causal ? min(2 * I + 2, nb64) : nb64;
+}
+
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
+  using L = Bwd64Smem;
+  constexpr int D = 128;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t bar0 = base + L::BARS;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1);
+  auto FULL_T = [&](int s) { return BAR(2 + s); };
+  auto EMPTY_T = [&](int s) { return BAR(4 + s); };
+  auto FULL_S = [&](int s) { return BAR(6 + s); };
+  auto EMPTY_S = [&](int s) { return BAR(10 + s); };
+  auto S_FULL = [&](int b) { return BAR(14 + b); };
+  auto S_EMPTY = [&](int b) { return BAR(16 + b); };
+  auto G_FULL = [&](int b) { return BAR(18 + b); };
+  auto G_EMPTY = [&](int b) { return BAR(20 + b); };
+  auto P_FULL = [&](int b) { return BAR(22 + b); };
+  auto P_EMPTY = [&](int b) { return BAR(24 + b); };
+  const uint32_t DXI_FULL = BAR(26), DXI_EMPTY = BAR(27), DRAIN = BAR(28);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
+
+  WaitCtl wc{p.status, abort_flag, p.timeout_ns};
+  constexpr uint32_t T_S = 0, T_DXI = 256, T_P = 384;
+
+  if (threadIdx.x == 0) {
+    mbar_init(FULL_I, 1);
+    mbar_init(EMPTY_I, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(FULL_T(s), 1);
+      mbar_init(EMPTY_T(s), 1);
+      mbar_init(S_FULL(s), 1);
+      mbar_init(S_EMPTY(s), 16);
+      mbar_init(G_FULL(s), 16);
+      mbar_init(G_EMPTY(s), 1);
+      mbar_init(P_FULL(s), 1);
+      mbar_init(P_EMPTY(s), 4);
+    }
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(FULL_S(s), 1);
+      mbar_init(EMPTY_S(s), 1);
+    }
+    mbar_init(DXI_FULL, 1);
+    mbar_init(DXI_EMPTY, 4);
+    mbar_init(DRAIN, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == BWD_MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == BWD_TMA_WARP) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      for (int s = 0; s < p.n_seg; ++s) {
+        tma_prefetch_desc(&p.seg[s].tm_t);
+        tma_prefetch_desc(&p.seg[s].tm_s);
+        tma_prefetch_desc(&p.seg[s].tm_t64);
+        tma_prefetch_desc(&p.seg[s].tm_s64);
+        tma_prefetch_desc(&p.seg[s].tm_dx);
+      }
+      uint32_t nI = 0, nJ = 0;
+      uint32_t armsT[2] = {0, 0}, armsS[4] = {0, 0, 0, 0};
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        const Unit U = decode_unit(p, u);
+        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+          const int I = pass_block(p, pp, pass);
+          if (!(ok = mbar_wait(EMPTY_I, (nI & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
+          mbar_arrive_expect_tx(FULL_I, 2 * L::TILE_I);
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, I * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, I * BM, U.h, U.b);
+          }
+          ++nI;
+          const int nT = n_col_tiles64(p, I);
+          for (int J = 0; J < nT; ++J) {
+            const int tt = nJ & 1, ts = nJ & 3;
+            if (!(ok = mbar_wait(EMPTY_T(tt), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_T(tt), L::TILE_J);
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+              tma_load_4d(base + L::XT_R + tt * L::TILE_J + b * L::BOX_J, &U.seg->tm_t64,
+                          FULL_T(tt), b * 64, J * BN64, U.h, U.b);
+            ++armsT[tt];
+            if (!(ok = mbar_wait(EMPTY_S(ts), ((nJ >> 2) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_S(ts), L::TILE_J);
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+              tma_load_4d(base + L::XS_R + ts * L::TILE_J + b * L::BOX_J, &U.seg->tm_s64,
+                          FULL_S(ts), b * 64, J * BN64, U.h, U.b);
+            ++armsS[ts];
+            ++nJ;
+          }
+        }
+      }
+      if (nI) mbar_wait_drain(FULL_I, (nI - 1) & 1, kDrainNs);
+      for (int s = 0; s < 2; ++s)
+        if (armsT[s]) mbar_wait_drain(FULL_T(s), (armsT[s] - 1) & 1, kDrainNs);
+      for (int s = 0; s < 4; ++s)
+        if (armsS[s]) mbar_wait_drain(FULL_S(s), (armsS[s] - 1) & 1, kDrainNs);
+    }
+    __syncwarp();
+  } else if (warp == BWD_MMA_WARP) {
+    // ------------------------------------------------------------ MMA
+    // The whole warp runs this loop (descriptor words stay warp-uniform); one
+    // elected lane issues the MMAs and commits.
+    {
+      const uint32_t lead = elect_leader();
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN64, 0, 0);
+      constexpr uint32_t IDESC_GX = idesc_bf16_f32(BM, D, 0, 1);    // A = G (K-major), B = X_s[J] (MN)
+      constexpr uint32_t IDESC_PT = idesc_bf16_f32(D, BN64, 1, 1);  // A = X_s[I]^T (MN), B = G (MN)
+      uint32_t nI = 0, nJ = 0, ns = 0, ng = 0, nrb = 0;
+      bool ok = true, issued = false;
+      // Low descriptor words of every operand buffer (all share the high word
+      // of an 8-row-group stride of 1024 B).  K-major operands step along K by
+      // 32 B inside a 128 B row and by one box across 64-column boxes; MN-major
+      // operands step by 2 KB (16 rows) and name the next 64-column box in LBO.
+      // (a buffer's word is the stage-0 word plus stage * size/16)
+      const uint32_t HI_1024 = sw128_desc_hi(1024);
+      const uint32_t dXtI_k = sw128_desc_lo(base + L::XT_I, 16);
+      const uint32_t dXsI_k = sw128_desc_lo(base + L::XS_I, 16);
+      const uint32_t dXsI_mn = sw128_desc_lo(base + L::XS_I, BOX);
+      const uint32_t dXtJ_k0 = sw128_desc_lo(base + L::XT_R, 16);
+      const uint32_t dXsJ_k0 = sw128_desc_lo(base + L::XS_R, 16);
+      const uint32_t dXsJ_mn0 = sw128_desc_lo(base + L::XS_R, L::BOX_J);
+      const uint32_t dG_k0 = sw128_desc_lo(base + L::G, 16);
+      const uint32_t dG_mn0 = sw128_desc_lo(base + L::G, BOX);
+      constexpr uint32_t J_STEP = L::TILE_J >> 4, G_STEP = L::G_BYTES >> 4;
+      // gradient MMAs of the tile whose student slot is `ts`; `first` starts dX_I
+      auto grad = [&](int ts, bool first) -> bool {
+        const int b = ng & 1;
+        const uint32_t par = (ng >> 1) & 1;
+        if (!mbar_wait_warp(G_FULL(b), par, wc, W_MMA_G_FULL)) return false;
+        if (!mbar_wait_warp(P_EMPTY(b), par ^ 1, wc, W_MMA_P_EMPTY)) return false;
+        if (first && !mbar_wait_warp(DXI_EMPTY, (nrb & 1) ^ 1, wc, W_MMA_DXI_EMPTY)) return false;
+        tc_fence_after();
+        const uint32_t g_k = dG_k0 + b * G_STEP, g_mn = dG_mn0 + b * G_STEP;
+        const uint32_t xsj = dXsJ_mn0 + ts * J_STEP;
+        // dX_I += G X_s[J]: M = i, N = c, K = j (64); K steps of 32 B (G) and 2 KB (X_s[J])
+#pragma unroll
+        for (int k = 0; k < BN64 / 16; ++k)
+          umma_bf16_w_lead(lead, tmem + T_DXI, g_k + k * 2, HI_1024, xsj + k * 128, HI_1024, IDESC_GX,
+                      (!first || k > 0) ? 1u : 0u);
+        // P^T = X_s[I]^T G: M = c, N = j, K = i (128); K steps of 2 KB in both
+#pragma unroll
+        for (int k = 0; k < BM / 16; ++k)
+          umma_bf16_w_lead(lead, tmem + T_P + b * 64, dXsI_mn + k * 128, HI_1024, g_mn + k * 128, HI_1024,
+                      IDESC_PT, k > 0 ? 1u : 0u);
+        umma_commit_lead(lead, G_EMPTY(b));
+        umma_commit_lead(lead, P_FULL(b));
+        umma_commit_lead(lead, EMPTY_S(ts));
+        ++ng;
+        return true;
+      };
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        (void)u;
+        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+          const int I = pass_block(p, pp, pass);
+          if (!(ok = mbar_wait_warp(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
+          const int nT = n_col_tiles64(p, I);
+          int prev_ts = -1;
+          for (int J = 0; J < nT; ++J) {
+            const int tt = nJ & 1, ts = nJ & 3, b = ns & 1;
+            if (!(ok = mbar_wait_warp(FULL_T(tt), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+            if (!(ok = mbar_wait_warp(S_EMPTY(b), ((ns >> 1) & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
+            tc_fence_after();
+            const uint32_t acc = tmem + T_S + b * 128;
+            const uint32_t xtj = dXtJ_k0 + tt * J_STEP, xsj = dXsJ_k0 + ts * J_STEP;
+            // K steps: 32 B within a 128 B row, then the next 64-column box
+            // (16 KB apart for 128-row tiles, 8 KB for 64-row tiles)
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k)
+              umma_bf16_w_lead(lead, acc, dXtI_k + (k >> 2) * (BOX >> 4) + (k & 3) * 2, HI_1024,
+                          xtj + (k >> 2) * (L::BOX_J >> 4) + (k & 3) * 2, HI_1024, IDESC_S,
+                          k > 0 ? 1u : 0u);
+            issued = true;
+            umma_commit_lead(lead, EMPTY_T(tt));
+            if (!(ok = mbar_wait_warp(FULL_S(ts), (nJ >> 2) & 1, wc, W_MMA_FULL_J))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k)
+              umma_bf16_w_lead(lead, acc + 64, dXsI_k + (k >> 2) * (BOX >> 4) + (k & 3) * 2, HI_1024,
+                          xsj + (k >> 2) * (L::BOX_J >> 4) + (k & 3) * 2, HI_1024, IDESC_S,
+                          k > 0 ? 1u : 0u);
+            umma_commit_lead(lead, S_FULL(b));
+            ++ns;
+            ++nJ;
+            if (prev_ts >= 0 && !(ok = grad(prev_ts, J == 1))) break;
+            prev_ts = ts;
+          }
+          if (!ok) break;
+          if (!(ok = grad(prev_ts, nT == 1))) break;
+          umma_commit_lead(lead, EMPTY_I);
+          umma_commit_lead(lead, DXI_FULL);
+          ++nI;
+          ++nrb;
+        }
+      }
+      if (issued) {
+        umma_commit_lead(lead, DRAIN);
+        mbar_wait_drain(DRAIN, 0, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= BWD_EPI_WARP) {
+    // ------------------------------------------------------- epilogue
+    const int q = warp - BWD_EPI_WARP;
+    const uint32_t stg = base + L::STG + q * 2 * L::STG_BYTES;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t np = 0, nrb = 0, nstg = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      const Unit U = decode_unit(p, u);
+      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+        const int I = pass_block(p, pp, pass);
+        const int nT = n_col_tiles64(p, I);
+        for (int J = 0; J < nT; ++J) {
+          const int b = np & 1;
+          ok = mbar_wait(P_FULL(b), (np >> 1) & 1, wc, W_EPI_P_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          // P^T rows are the d columns c = 32q + lane; its columns are the 64
+          // rows j of column tile J.  Each 32-row half becomes one 32 x 32 box
+          // of dX[J] (row j, column c), written one 128-byte row per store.
+#pragma unroll 1
+          for (int jb = 0; jb < 2; ++jb) {
+            float v[32];
+            tmem_ld32(tmem + lane_addr + T_P + b * 64 + jb * 32, v);
+            tmem_wait_ld();
+            if (jb == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(P_EMPTY(b));
+            }
+            const uint32_t buf = stg + (nstg & 1) * L::STG_BYTES;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              st_shared_b32(buf + jj * 128 + (((lane >> 2) ^ (jj & 7)) << 4) + (lane & 3) * 4,
+                            v[jj]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int row0 = J * BN64 + jb * 32;
+            if (lane == 0) {
+              if (row0 < p.N) tma_reduce_add_4d(&U.seg->tm_dx, buf, q * 32, row0, U.h, U.b);
+              bulk_commit();
+            }
+            ++nstg;
+          }
+          ++np;
+        }
+        if (!ok) break;
+        ok = mbar_wait(DXI_FULL, nrb & 1, wc, W_EPI_DXI_FULL);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        epilogue_reduce<D>(tmem + lane_addr + T_DXI, stg, nstg, &U.seg->tm_dx, I * BM + q * 32,
+                           U.h, U.b, p.N, lane, DXI_EMPTY);
+        ++nrb;
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  } else {
+    // --------------------------------------------------- row warpgroups
+    const int q = warp & 3;
+    const int wg = warp >> 2;      // 16-column slice of each 64-column tile
+    const int r = q * 32 + lane;
+    const float sl2 = p.sl2;
+    const uint32_t row_g = r * 128;  // row r of a G buffer: 128 bytes, chunks 2wg, 2wg+1
+    uint32_t ns = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      const Unit U = decode_unit(p, u);
+      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
+        const int I = pass_block(p, pp, pass);
+        const int row = I * BM + r;
+        const bool rvalid = row < p.N;
+        float bt = 0.f, bs = 0.f, mul = 0.f;
+        if (rvalid) {
+          const float4 st4 = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + row];
+          bt = -st4.y * kLog2e;
+          bs = -st4.z * kLog2e;
+          const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(p.N);
+          mul = up * p.scale;   // the logit scale of dX_s is folded into G
+        }
+        const int lim = !rvalid ? -1 : (p.causal ? min(row, p.N - 1) : p.N - 1);
+        const int nT = n_col_tiles64(p, I);
+        const float2 sl2v = make_float2(sl2, sl2), btv = make_float2(bt, bt),
+                     bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
+                     m1 = make_float2(-1.f, -1.f);
+        for (int J = 0; J < nT; ++J) {
+          const int b = ns & 1;
+          const uint32_t par = (ns >> 1) & 1;
+          ok = mbar_wait(S_FULL(b), par, wc, W_SM_S_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + T_S + b * 128 + wg * 16;
+          float t[16], s[16];
+          tmem_ld16(ta, t);
+          tmem_ld16(ta + 64, s);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(S_EMPTY(b));
+          const int col0 = J * BN64 + wg * 16;
+          const bool need_mask = !rvalid || (col0 + 15 > lim);
+          uint32_t pk[8];
+#pragma unroll
+          for (int k = 0; k < 16; k += 2) {
+            const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
+            const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
+            float2 et, es;
+            if (bwd_poly_pair(k >> 1)) {
+              et = exp2_poly2<3>(at);
+              es = exp2_poly2<3>(as);
+            } else {
+              et = ex2_approx2(at);
+              es = ex2_approx2(as);
+            }
+            float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
+            if (need_mask) {
+              g.x = (col0 + k <= lim) ? g.x : 0.f;
+              g.y = (col0 + k + 1 <= lim) ? g.y : 0.f;
+            }
+            pk[k >> 1] = pack_bf16x2(g.x, g.y);
+          }
+          ok = mbar_wait(G_EMPTY(b), par ^ 1, wc, W_SM_G_EMPTY);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          const uint32_t gsm = base + L::G + b * L::G_BYTES + row_g;
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int cc = 2 * wg + h2;
+            st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[4 * h2], pk[4 * h2 + 1], pk[4 * h2 + 2],
+                         pk[4 * h2 + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(G_FULL(b));
+          ++ns;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == BWD_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -805,11 +1290,17 @@ cudaError_t tc_launch_fwd(const TcParams& p, int d, int grid, cudaStream_t strea
 }
 
 cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t stream) {
-  return d == 64 ? launch_bwd<64>(p, grid, stream) : launch_bwd<128>(p, grid, stream);
+  if (d == 64) return launch_bwd<64>(p, grid, stream);
+  cudaError_t e = cudaFuncSetAttribute(relkl_bwd_tc64_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Bwd64Smem::ALLOC);
+  if (e != cudaSuccess) return e;
+  relkl_bwd_tc64_kernel<<<grid, BWD_THREADS, Bwd64Smem::ALLOC, stream>>>(p);
+  return cudaGetLastError();
 }
 
 size_t tc_smem_bytes(int d, int is_bwd) {
-  if (is_bwd) return d == 64 ? BwdSmem<64>::ALLOC : BwdSmem<128>::ALLOC;
+  if (is_bwd) return d == 64 ? BwdSmem<64>::ALLOC : Bwd64Smem::ALLOC;
   return d == 64 ? FwdSmem<64>::ALLOC : FwdSmem<128>::ALLOC;
 }
 

@@ -210,6 +210,7 @@ def main():
 
     import torch.distributed as dist
     import attention_relation_kl_b200 as rk
+    from attention_relation_kl_b200.replicas import max_over_ranks, replica_seed
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -227,7 +228,7 @@ def main():
         torch.cuda.synchronize()
 
     # inputs: this rank's replica (seed offset by rank), resident in HBM
-    wr = workload.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
+    wr = workload.Workload(**{**w.__dict__, "seed": replica_seed(w.seed, rank)})
     t_gen = time.perf_counter()
     x = workload.generate(wr)
     t_gen = time.perf_counter() - t_gen
@@ -279,10 +280,7 @@ def main():
     code, where = rk.relkl_get_device_error(ws)
     if code != 0:
         raise SystemExit(f"device wait ran out in the timed region (site {where})")
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     peak_alloc = torch.cuda.max_memory_allocated(dev)
 
     # end to end through the public API with host buffers
@@ -308,11 +306,7 @@ def main():
                 hd.copy_(dv, non_blocking=True)
         e1.record(stream)
         barrier()
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
 
     fl_fwd, fl_bwd = flops(w)
     total_fl = (fl_fwd + fl_bwd) * world

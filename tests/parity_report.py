@@ -1,0 +1,101 @@
+"""Parity margins of the CUDA path against the float64 oracle, as a table.
+
+    python tests/parity_report.py [--full] > parity.md
+
+For each case: the worst per-row KL error as a fraction of its tolerance
+(1e-3 |kl| + 1e-6), the relative error of the total KL, and the max-norm
+relative dX error against its tolerance (2e-2 for bf16 inputs, 2e-4 for the
+fp32 path).  --full adds the workload-sized cases (sampled units and rows),
+which take a few minutes of oracle time.  Needs a CUDA device.
+"""
+import os
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+import attention_relation_kl_b200 as rk  # noqa: E402
+import workload  # noqa: E402
+from oracle import dense  # noqa: E402
+from parity import DX_TOL_BF16, DX_TOL_FP32, KL_ATOL, KL_RTOL, to_np  # noqa: E402
+
+
+def margins(kl, ref_kl, dx, ref_dx, dx_tol):
+    kl, ref_kl = np.asarray(kl, np.float64), np.asarray(ref_kl, np.float64)
+    kl_frac = float(np.max(np.abs(kl - ref_kl) / (KL_RTOL * np.abs(ref_kl) + KL_ATOL)))
+    tot = float(abs(kl.sum() - ref_kl.sum()) / max(abs(ref_kl.sum()), 1e-30))
+    dx_rel = float(np.max(np.abs(dx - ref_dx)) / max(np.max(np.abs(ref_dx)), 1e-30))
+    return kl_frac, tot, dx_rel, dx_rel / dx_tol
+
+
+def small_cases():
+    cases = []
+    for (N, d, causal, B, H, dtype) in [(128, 128, True, 1, 1, "bf16"), (300, 64, True, 1, 2, "bf16"),
+                                        (1000, 128, True, 1, 1, "bf16"), (513, 64, False, 1, 1, "bf16"),
+                                        (256, 64, True, 1, 1, "fp32"), (200, 96, True, 1, 2, "bf16")]:
+        w = workload.tiny_custom(N=N, d=d, dtype=dtype, seed=N + d, causal=causal, B=B, H=H)
+        xt, xs = workload.generate(w)["q"]
+        cases.append((f"Q/Q RoPE PI4x N={N} d={d} {'causal' if causal else 'full'} {dtype}",
+                      xt, xs, causal))
+    xt, xs = workload.gaussian_pair((1, 2, 640, 128), seed=5, noise=0.05, dtype=torch.bfloat16)
+    cases.append(("V/V sigma=0.05 N=640 d=128 bf16", xt, xs, True))
+    return cases
+
+
+def run_small(out):
+    for name, xt, xs, causal in small_cases():
+        gt, gs = xt.cuda(), xs.cuda()
+        path = "tcgen05" if rk.relkl_path_for(gt, causal) == 1 else "CUDA-core fp32"
+        kl, st = rk.relkl_fwd(gt, gs, causal)
+        dx = rk.relkl_bwd(gt, gs, st, None, causal)
+        torch.cuda.synchronize()
+        tol = DX_TOL_BF16 if path == "tcgen05" else DX_TOL_FP32
+        m = margins(to_np(kl), dense.fwd(xt, xs, causal)["kl"], to_np(dx),
+                    dense.bwd(xt, xs, None, causal), tol)
+        out.append((name, path, "all rows", *m))
+
+
+def run_full(out):
+    for cfg, units in (("llama2_h32_n4k", [("q", 0, 0), ("v", 0, 31)]),
+                       ("gqa_llama3_n16k", [("k", 0, 3), ("v", 1, 7)]),
+                       ("ext_h32_n32k", [("q", 0, 0), ("v", 0, 31)])):
+        w = workload.get_config(cfg)
+        x = workload.generate(w)
+        pairs = [(x[r][0].cuda(), x[r][1].cuda()) for r in w.relations]
+        outs = rk.relkl_fwd_qkv(pairs, w.causal)
+        dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal)
+        torch.cuda.synchronize()
+        ri = {r: i for i, r in enumerate(w.relations)}
+        for rel, b, h in units:
+            xt, xs = x[rel][0][b, h], x[rel][1][b, h]
+            ref = dense.fwd_unit(xt, xs, w.causal)
+            rows = [0, 1, 127, 128, w.N // 2, w.N - 1]
+            ref_dx = dense.bwd_rows(xt, xs, rows, causal=w.causal, lse=ref)
+            m = margins(to_np(outs[ri[rel]][0][b, h]), ref["kl"],
+                        to_np(dxs[ri[rel]][b, h])[rows], ref_dx, DX_TOL_BF16)
+            out.append((f"{cfg} unit ({rel}, b={b}, h={h})", "tcgen05 fused QKV",
+                        f"kl all {w.N} rows, dX rows {rows}", *m))
+
+
+def main():
+    out = []
+    t0 = time.time()
+    run_small(out)
+    if "--full" in sys.argv:
+        run_full(out)
+    print(f"# Parity margins against the float64 oracle ({torch.cuda.get_device_name(0)})\n")
+    print("Fractions are of the tolerance: < 1 passes.\n")
+    print("| case | path | compared | worst kl err / tol | total kl rel err | dX max-norm rel err | dX err / tol |")
+    print("|---|---|---|---|---|---|---|")
+    for name, path, cmp, klf, tot, dxr, dxf in out:
+        print(f"| {name} | {path} | {cmp} | {klf:.3f} | {tot:.2e} | {dxr:.2e} | {dxf:.3f} |")
+    print(f"\n({time.time() - t0:.0f} s)")
+
+
+if __name__ == "__main__":
+    main()
