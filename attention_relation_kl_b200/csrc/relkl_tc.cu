@@ -318,105 +318,97 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
           if (!ok) break;
           tc_fence_after();
           const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * 256 + wg * 32;
-          // two 16-column halves: fewer live registers, more exps in flight.  The
-          // TMEM buffer is handed back after the second load (the MMA warp only
-          // needs it again two tiles later).
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            float t[16], s[16];
-            tmem_ld16(ta + hh * 16, t);
-            tmem_ld16(ta + 128 + hh * 16, s);
-            tmem_wait_ld();
-            if (hh == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(TE(buf));
+          float t[32], s[32];
+          tmem_ld32(ta, t);
+          tmem_ld32(ta + 128, s);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(TE(buf));
+          ++nt;
+          const int col0 = J * BN + wg * 32;
+          const bool need_mask = (p.causal && J == I) || (col0 + 32 > p.N);
+          if (!need_mask) {
+            float m4[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) m4[k] = fmaxf(t[k], s[k]);
+#pragma unroll
+            for (int k = 4; k < 32; ++k) m4[k & 3] = fmaxf(m4[k & 3], fmaxf(t[k], s[k]));
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            if (mx > m_run) {
+              const float a = ex2_approx((m_run - mx) * sl2);
+              const float2 a2 = make_float2(a, a);
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                S2[k] = __fmul2_rn(S2[k], a2);
+                C2[k] = __fmul2_rn(C2[k], a2);
+                A2[k] = __fmul2_rn(A2[k], a2);
+              }
+              m_run = mx;
             }
-            const int col0 = J * BN + wg * 32 + hh * 16;
-            const bool need_mask = (p.causal && J == I) || (col0 + 16 > p.N);
-            if (!need_mask) {
-              float m4[4];
+            const float nb = -m_run * sl2;
+            const float2 sl2v = make_float2(sl2, sl2), nbv = make_float2(nb, nb);
+            const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
-              for (int k = 0; k < 4; ++k) m4[k] = fmaxf(t[k], s[k]);
-#pragma unroll
-              for (int k = 4; k < 16; ++k) m4[k & 3] = fmaxf(m4[k & 3], fmaxf(t[k], s[k]));
-              const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-              if (mx > m_run) {
-                const float a = ex2_approx((m_run - mx) * sl2);
-                const float2 a2 = make_float2(a, a);
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                  S2[k] = __fmul2_rn(S2[k], a2);
-                  C2[k] = __fmul2_rn(C2[k], a2);
-                  A2[k] = __fmul2_rn(A2[k], a2);
-                }
-                m_run = mx;
+            for (int k = 0; k < 32; k += 2) {
+              const float2 tv = make_float2(t[k], t[k + 1]);
+              const float2 sv = make_float2(s[k], s[k + 1]);
+              const float2 at = __ffma2_rn(tv, sl2v, nbv);
+              const float2 as = __ffma2_rn(sv, sl2v, nbv);
+              float2 et, es;
+              if (fwd_poly_pair(k >> 1)) {
+                et = exp2_poly2<5>(at);
+                es = exp2_poly2<5>(as);
+              } else {
+                et = ex2_approx2(at);
+                es = ex2_approx2(as);
               }
+              const int a = (k >> 1) & 1;
+              S2[a] = __fadd2_rn(S2[a], et);
+              C2[a] = __fadd2_rn(C2[a], __ffma2_rn(et, m1, es));
+              A2[a] = __ffma2_rn(et, __ffma2_rn(sv, m1, tv), A2[a]);
+            }
+          } else {
+            // diagonal or ragged tile: per-entry predicate
+            const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (col0 + k <= lim) mx = fmaxf(mx, fmaxf(t[k], s[k]));
+            if (mx > m_run) {
+              const float a = ex2_approx((m_run - mx) * sl2);
+              const float2 a2 = make_float2(a, a);
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                S2[k] = __fmul2_rn(S2[k], a2);
+                C2[k] = __fmul2_rn(C2[k], a2);
+                A2[k] = __fmul2_rn(A2[k], a2);
+              }
+              m_run = mx;
+            }
+            if (m_run > -INFINITY) {
               const float nb = -m_run * sl2;
-              const float2 sl2v = make_float2(sl2, sl2), nbv = make_float2(nb, nb);
-              const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
-              for (int k = 0; k < 16; k += 2) {
-                const float2 tv = make_float2(t[k], t[k + 1]);
-                const float2 sv = make_float2(s[k], s[k + 1]);
-                const float2 at = __ffma2_rn(tv, sl2v, nbv);
-                const float2 as = __ffma2_rn(sv, sl2v, nbv);
-                float2 et, es;
-                if (fwd_poly_pair(k >> 1)) {
-                  et = exp2_poly2<5>(at);
-                  es = exp2_poly2<5>(as);
-                } else {
-                  et = ex2_approx2(at);
-                  es = ex2_approx2(as);
-                }
-                const int a = (k >> 1) & 1;
-                S2[a] = __fadd2_rn(S2[a], et);
-                C2[a] = __fadd2_rn(C2[a], __ffma2_rn(et, m1, es));
-                A2[a] = __ffma2_rn(et, __ffma2_rn(sv, m1, tv), A2[a]);
-              }
-            } else {
-              // diagonal or ragged tile: per-entry predicate
-              const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;  // last allowed column
-              float mx = -INFINITY;
-#pragma unroll
-              for (int k = 0; k < 16; ++k)
-                if (col0 + k <= lim) mx = fmaxf(mx, fmaxf(t[k], s[k]));
-              if (mx > m_run) {
-                const float a = ex2_approx((m_run - mx) * sl2);
-                const float2 a2 = make_float2(a, a);
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                  S2[k] = __fmul2_rn(S2[k], a2);
-                  C2[k] = __fmul2_rn(C2[k], a2);
-                  A2[k] = __fmul2_rn(A2[k], a2);
-                }
-                m_run = mx;
-              }
-              if (m_run > -INFINITY) {
-                const float nb = -m_run * sl2;
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                  if (col0 + k <= lim) {
-                    const float et = ex2_approx(fmaf(t[k], sl2, nb));
-                    const float es = ex2_approx(fmaf(s[k], sl2, nb));
-                    float2& Sa = S2[(k >> 1) & 1];
-                    float2& Ca = C2[(k >> 1) & 1];
-                    float2& Aa = A2[(k >> 1) & 1];
-                    if (k & 1) {
-                      Sa.y += et;
-                      Ca.y += es - et;
-                      Aa.y = fmaf(et, t[k] - s[k], Aa.y);
-                    } else {
-                      Sa.x += et;
-                      Ca.x += es - et;
-                      Aa.x = fmaf(et, t[k] - s[k], Aa.x);
-                    }
+              for (int k = 0; k < 32; ++k) {
+                if (col0 + k <= lim) {
+                  const float et = ex2_approx(fmaf(t[k], sl2, nb));
+                  const float es = ex2_approx(fmaf(s[k], sl2, nb));
+                  float2& Sa = S2[(k >> 1) & 1];
+                  float2& Ca = C2[(k >> 1) & 1];
+                  float2& Aa = A2[(k >> 1) & 1];
+                  if (k & 1) {
+                    Sa.y += et;
+                    Ca.y += es - et;
+                    Aa.y = fmaf(et, t[k] - s[k], Aa.y);
+                  } else {
+                    Sa.x += et;
+                    Ca.x += es - et;
+                    Aa.x = fmaf(et, t[k] - s[k], Aa.x);
                   }
                 }
               }
             }
           }
-          ++nt;
         }
         if (!ok) break;
         const float Sx = (S2[0].x + S2[0].y) + (S2[1].x + S2[1].y);
@@ -873,7 +865,7 @@ struct Bwd64Smem {
   static constexpr int STG_BYTES = 32 * 32 * 4;
   static constexpr int BARS = STG + 4 * 2 * STG_BYTES;
   // full_I, empty_I, fullT[2], emptyT[2], fullS[4], emptyS[4], s_full[2], s_empty[2],
-  // g_full[2], g_empty[2], p_full[2], p_empty[2], dxi_full, dxi_empty, drain
+  // g_full[2], (2 spare), p_full[2], p_empty[2], dxi_full, dxi_empty, drain
   static constexpr int NBAR = 31;
   static constexpr int MISC = BARS + NBAR * 8;
   static constexpr int BYTES = MISC + 16;
@@ -910,7 +902,6 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
   auto S_FULL = [&](int b) { return BAR(14 + b); };
   auto S_EMPTY = [&](int b) { return BAR(16 + b); };
   auto G_FULL = [&](int b) { return BAR(18 + b); };
-  auto G_EMPTY = [&](int b) { return BAR(20 + b); };
   auto P_FULL = [&](int b) { return BAR(22 + b); };
   auto P_EMPTY = [&](int b) { return BAR(24 + b); };
   const uint32_t DXI_FULL = BAR(26), DXI_EMPTY = BAR(27), DRAIN = BAR(28);
@@ -929,7 +920,6 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
       mbar_init(S_FULL(s), 1);
       mbar_init(S_EMPTY(s), 16);
       mbar_init(G_FULL(s), 16);
-      mbar_init(G_EMPTY(s), 1);
       mbar_init(P_FULL(s), 1);
       mbar_init(P_EMPTY(s), 4);
     }
@@ -1052,7 +1042,6 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
         for (int k = 0; k < BM / 16; ++k)
           umma_bf16_w_lead(lead, tmem + T_P + b * 64, dXsI_mn + k * 128, HI_1024, g_mn + k * 128, HI_1024,
                       IDESC_PT, k > 0 ? 1u : 0u);
-        umma_commit_lead(lead, G_EMPTY(b));
         umma_commit_lead(lead, P_FULL(b));
         umma_commit_lead(lead, EMPTY_S(ts));
         ++ng;
@@ -1237,9 +1226,10 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
             }
             pk[k >> 1] = pack_bf16x2(g.x, g.y);
           }
-          ok = mbar_wait(G_EMPTY(b), par ^ 1, wc, W_SM_G_EMPTY);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
+          // No wait for G buffer b: the MMA warp issues the gradient MMAs of tile
+          // t-2 (the last reader of this buffer) before the logit MMAs of tile t,
+          // and the commit behind S_FULL covers every MMA it issued before, so
+          // having seen S_FULL(t) the buffer is free.
           const uint32_t gsm = base + L::G + b * L::G_BYTES + row_g;
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
