@@ -190,6 +190,65 @@ def run_reference(args, w):
     return 0
 
 
+# ----------------------------------------------------------- N sweep (one GPU)
+
+def run_sweep(args):
+    """Throughput and memory over N at fixed B*N (the scaling/roofline workload).
+
+    Extra memory = peak allocated during fwd+bwd minus the inputs and dX: the
+    O(N) row statistics.  A materialised relation would add 4*N*N bytes per unit.
+    """
+    import attention_relation_kl_b200 as rk
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ws = rk.workspace(dev)
+    for N in workload.SWEEP_N:
+        w = workload.sweep_config(N)
+        x = workload.generate(w)
+        pairs = [(x[r][0].to(dev), x[r][1].to(dev)) for r in w.relations]
+        del x
+        in_bytes = sum(a.numel() * a.element_size() * 2 for a, _ in pairs)
+        dxs = [torch.empty(a.shape, dtype=torch.float32, device=dev) for a, _ in pairs]
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        outs = rk.relkl_fwd_qkv(pairs, w.causal, ws=ws)
+        rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
+        torch.cuda.synchronize()
+        extra = torch.cuda.max_memory_allocated(dev) - base
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        for _ in range(2):
+            rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
+            rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
+        torch.cuda.synchronize()
+        fwd_ms = bwd_ms = 0.0
+        steps = max(1, args.steps)
+        for _ in range(steps):
+            ev[0].record()
+            rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
+            ev[1].record()
+            rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
+            ev[2].record()
+            torch.cuda.synchronize()
+            fwd_ms += ev[0].elapsed_time(ev[1]) / steps
+            bwd_ms += ev[1].elapsed_time(ev[2]) / steps
+        code, where = rk.relkl_get_device_error(ws)
+        fl_f, fl_b = flops(w)
+        rows = w.B * w.N * sum(w.heads(r) for r in w.relations)
+        print(json.dumps({
+            "sweep": w.name, "N": N, "B": w.B, "units": w.n_units,
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "fwd_tflops": fl_f / fwd_ms / 1e9, "bwd_tflops": fl_b / bwd_ms / 1e9,
+            "total_tflops": (fl_f + fl_b) / (fwd_ms + bwd_ms) / 1e9,
+            "tokens_per_s": w.B * w.N / ((fwd_ms + bwd_ms) * 1e-3),
+            "inputs_bytes": in_bytes, "dx_bytes": sum(d.numel() * 4 for d in dxs),
+            "extra_bytes": extra, "extra_bytes_per_row": extra / rows,
+            "dense_relation_bytes_per_unit": 4 * N * N, "device_status": code}), flush=True)
+        del pairs, dxs, outs
+        torch.cuda.empty_cache()
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def main():
@@ -202,11 +261,16 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--ref-prefix", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="sequence-length sweep (B*N = 65536): one JSON line per N with "
+                         "throughput and peak extra memory, instead of the bench line")
     args = ap.parse_args()
     w = workload.get_config(args.config)
 
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.sweep:
+        return run_sweep(args)
 
     import torch.distributed as dist
     import attention_relation_kl_b200 as rk
@@ -319,7 +383,7 @@ def main():
     bwd_avg = sum(bwd_ms) / len(bwd_ms)
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
     achieved = fl_bwd / (bwd_avg * 1e-3) / 1e12
-    traffic = traffic_record("relkl_bwd_tc_kernel")
+    traffic = traffic_record("relkl_bwd_tc64_kernel" if w.d == 128 else "relkl_bwd_tc_kernel")
 
     result = None
     if rank == 0:
@@ -340,7 +404,8 @@ def main():
             "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
             "fwd_tflops": fl_fwd / (fwd_avg * 1e-3) / 1e12,
             "bwd_tflops": fl_bwd / (bwd_avg * 1e-3) / 1e12,
-            "roofline": {"kernel": "relkl_bwd_tc_kernel", "bound": "tensor", "achieved": achieved,
+            "roofline": {"kernel": "relkl_bwd_tc64_kernel" if w.d == 128 else "relkl_bwd_tc_kernel",
+                         "bound": "tensor", "achieved": achieved,
                          "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
                          "traffic": traffic,
                          "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",

@@ -174,7 +174,9 @@ def _sampled(w: workload.Workload, units, dx_units, n_dx_rows=6):
         xt, xs = x[rel][0][b, h], x[rel][1][b, h]
         kl, st = outs[rel_idx[rel]]
         full = (rel, b, h) in dx_units
-        ref = dense.fwd_unit(xt, xs, w.causal) if full else dense.fwd_rows(xt, xs, rows, w.causal)
+        slab = 2048 if N <= 32768 else 512
+        ref = (dense.fwd_unit(xt, xs, w.causal, slab=slab) if full
+               else dense.fwd_rows(xt, xs, rows, w.causal))
         sel = slice(None) if full else rows
         assert_kl(to_np(kl[b, h])[sel], ref["kl"], what=f"kl[{rel},{b},{h}]")
         assert_stats(to_np(st[b, h])[sel], ref)
@@ -201,3 +203,10 @@ def test_config_ext_h32_n32k():
     w = workload.CONFIGS["ext_h32_n32k"]
     units = [("q", 0, 0), ("k", 0, 17), ("v", 0, 31)]
     _sampled(w, units, dx_units={("q", 0, 0)})
+
+
+def test_config_sweep_n64k():
+    # the largest point of the sequence-length sweep: B=1, H=32, N=65536
+    w = workload.sweep_config(65536)
+    units = [("q", 0, 0), ("k", 0, 9), ("v", 0, 31)]
+    _sampled(w, units, dx_units={("k", 0, 9)})
