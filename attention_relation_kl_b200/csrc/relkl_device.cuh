@@ -395,5 +395,4 @@ __device__ __forceinline__ void st_shared_b32(uint32_t addr, float v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(__float_as_uint(v)) : "memory");
 }
 
-
 }  // namespace relkl

@@ -1254,6 +1254,491 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
   }
 }
 
+// =========================================================================
+//        BACKWARD, d = 128: adjacent row-block pairs, column-tile outer
+// =========================================================================
+// The same mathematics again, scheduled so that the column-side product
+// P^T = sum_i X_s[i]^T G[i, J] of a 64-column tile J is summed over 256 rows
+// (two adjacent 128-row blocks R0 = 2k, R1 = 2k+1) in TMEM before it is added
+// into dX once.  Against one 128-row block per pass this halves the f32
+// reduce-adds into dX (an L2-throughput cost) and the column-tile loads per
+// logit.  Tiles run in the order (R0, J), (R1, J), (R0, J+1), ...; column
+// tiles that only R1 reaches under the causal mask run alone.  Two warps
+// issue MMAs: one the logits of the next tile, one the gradient products of
+// the tile whose G was just stored.
+//   TMEM: Z_t/Z_s 0..127 (one buffer: the row warps read all of it at once
+//         and release it), dX_R0 128..255, dX_R1 256..383, P^T 2 x 64 at 384.
+//   smem: X_t, X_s of R0 and R1 (4 x 32 KB); teacher and student column
+//         rings 2 x 16 KB each; G 16 KB; epilogue staging 4 x 4 KB.
+// A work item is the pair sequence k = npb-1-m followed by k = m (npb row-block
+// pairs per unit), which evens out the causal triangle across items.  With
+// few row blocks the items are too coarse to balance 148 SMs, so sequences of
+// at most 32 row blocks use relkl_bwd_tc64_kernel instead.
+struct BwdPairSmem {
+  static constexpr int TILE_I = BM * 128 * 2;        // 128 rows: boxes of 128 x 64 (16 KB)
+  static constexpr int BOX_I = BM * 128;
+  static constexpr int TILE_J = 64 * 128 * 2;        // 64 rows: boxes of 64 x 64 (8 KB)
+  static constexpr int BOX_J = 64 * 128;
+  static constexpr int XT_R0 = 0;
+  static constexpr int XS_R0 = TILE_I;
+  static constexpr int XT_R1 = 2 * TILE_I;
+  static constexpr int XS_R1 = 3 * TILE_I;
+  static constexpr int XT_J = 4 * TILE_I;            // 2 stages
+  static constexpr int XS_J = XT_J + 2 * TILE_J;     // 2 stages
+  static constexpr int G = XS_J + 2 * TILE_J;        // 128 x 64 bf16
+  static constexpr int G_BYTES = BM * 64 * 2;
+  static constexpr int STG = G + G_BYTES;            // 4 warps x one 32 x 32 f32 box
+  static constexpr int STG_BYTES = 32 * 32 * 4;
+  static constexpr int BARS = STG + 4 * STG_BYTES;
+  // full_I, empty_I, fullT[2], emptyT[2], fullS[2], emptyS[2], s_full, s_empty,
+  // g_full, g_empty, p_full[2], p_empty[2], dxi_full, dxi_empty, drain x 2
+  static constexpr int NBAR = 22;
+  static constexpr int MISC = BARS + NBAR * 8;
+  static constexpr int BYTES = MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+};
+static_assert(BwdPairSmem::ALLOC <= 232448, "backward shared memory exceeds 227 KB");
+// warps 0-15 row, 16-19 epilogue, 20 TMA, 21 logit MMAs, 22 gradient MMAs
+constexpr int BWDP_THREADS = 736;
+// smallest row-block count (N > 4096) that takes the pair kernel
+constexpr int kPairMinBlocks = 33;
+constexpr int BWDP_LOGIT_WARP = 21, BWDP_GRAD_WARP = 22;
+
+// Sequence `which` (0 or 1) of pair item m: its first row block, or -1.
+__device__ __forceinline__ int pair_seq_block(const TcParams& p, int m, int which) {
+  const int npb = (p.nblk + 1) / 2;
+  const int k = which == 0 ? npb - 1 - m : m;
+  if (which == 1 && k == npb - 1 - m) return -1;
+  return 2 * k;
+}
+
+__global__ void __launch_bounds__(BWDP_THREADS, 1)
+relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
+  using L = BwdPairSmem;
+  constexpr int D = 128;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t bar0 = base + L::BARS;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1);
+  auto FULL_T = [&](int s) { return BAR(2 + s); };
+  auto EMPTY_T = [&](int s) { return BAR(4 + s); };
+  auto FULL_S = [&](int s) { return BAR(6 + s); };
+  auto EMPTY_S = [&](int s) { return BAR(8 + s); };
+  const uint32_t S_FULL = BAR(10), S_EMPTY = BAR(11), G_FULL = BAR(12), G_EMPTY = BAR(13);
+  auto P_FULL = [&](int b) { return BAR(14 + b); };
+  auto P_EMPTY = [&](int b) { return BAR(16 + b); };
+  const uint32_t DXI_FULL = BAR(18), DXI_EMPTY = BAR(19), DRAIN_L = BAR(20), DRAIN_G = BAR(21);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
+
+  WaitCtl wc{p.status, abort_flag, p.timeout_ns};
+  constexpr uint32_t T_S = 0, T_DX0 = 128, T_P = 384;
+
+  if (threadIdx.x == 0) {
+    mbar_init(FULL_I, 1);
+    mbar_init(EMPTY_I, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(FULL_T(s), 1);
+      mbar_init(EMPTY_T(s), 1);
+      mbar_init(P_FULL(s), 1);
+      mbar_init(P_EMPTY(s), 4);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(FULL_S(s), 1);
+      mbar_init(EMPTY_S(s), 1);
+    }
+    mbar_init(S_FULL, 1);
+    mbar_init(S_EMPTY, 16);
+    mbar_init(G_FULL, 16);
+    mbar_init(G_EMPTY, 1);
+    mbar_init(DXI_FULL, 1);
+    mbar_init(DXI_EMPTY, 4);
+    mbar_init(DRAIN_L, 1);
+    mbar_init(DRAIN_G, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == BWDP_LOGIT_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int ipu = p.n_pairs;   // pair items per unit
+
+  if (warp == BWD_TMA_WARP) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      for (int s = 0; s < p.n_seg; ++s) {
+        tma_prefetch_desc(&p.seg[s].tm_t);
+        tma_prefetch_desc(&p.seg[s].tm_s);
+        tma_prefetch_desc(&p.seg[s].tm_t64);
+        tma_prefetch_desc(&p.seg[s].tm_s64);
+        tma_prefetch_desc(&p.seg[s].tm_dx);
+      }
+      uint32_t nseq = 0, nJ = 0;
+      uint32_t armsT[2] = {0, 0}, armsS[2] = {0, 0};
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int u = item / ipu, m = item - u * ipu;
+        const Unit U = decode_unit(p, u);
+        for (int w = 0; ok && w < 2; ++w) {
+          const int R0 = pair_seq_block(p, m, w);
+          if (R0 < 0) break;
+          const bool has1 = R0 + 1 < p.nblk;
+          if (!(ok = mbar_wait(EMPTY_I, (nseq & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
+          mbar_arrive_expect_tx(FULL_I, (has1 ? 4 : 2) * L::TILE_I);
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            tma_load_4d(base + L::XT_R0 + b * L::BOX_I, &U.seg->tm_t, FULL_I, b * 64, R0 * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_R0 + b * L::BOX_I, &U.seg->tm_s, FULL_I, b * 64, R0 * BM, U.h, U.b);
+            if (has1) {
+              tma_load_4d(base + L::XT_R1 + b * L::BOX_I, &U.seg->tm_t, FULL_I, b * 64, (R0 + 1) * BM,
+                          U.h, U.b);
+              tma_load_4d(base + L::XS_R1 + b * L::BOX_I, &U.seg->tm_s, FULL_I, b * 64, (R0 + 1) * BM,
+                          U.h, U.b);
+            }
+          }
+          ++nseq;
+          const int nT = n_col_tiles64(p, has1 ? R0 + 1 : R0);
+          for (int J = 0; J < nT; ++J) {
+            const int tt = nJ & 1, ts = nJ & 1;
+            if (!(ok = mbar_wait(EMPTY_T(tt), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_T(tt), L::TILE_J);
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+              tma_load_4d(base + L::XT_J + tt * L::TILE_J + b * L::BOX_J, &U.seg->tm_t64, FULL_T(tt),
+                          b * 64, J * BN64, U.h, U.b);
+            ++armsT[tt];
+            if (!(ok = mbar_wait(EMPTY_S(ts), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_S(ts), L::TILE_J);
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+              tma_load_4d(base + L::XS_J + ts * L::TILE_J + b * L::BOX_J, &U.seg->tm_s64, FULL_S(ts),
+                          b * 64, J * BN64, U.h, U.b);
+            ++armsS[ts];
+            ++nJ;
+          }
+        }
+      }
+      if (nseq) mbar_wait_drain(FULL_I, (nseq - 1) & 1, kDrainNs);
+      for (int s = 0; s < 2; ++s)
+        if (armsT[s]) mbar_wait_drain(FULL_T(s), (armsT[s] - 1) & 1, kDrainNs);
+      for (int s = 0; s < 2; ++s)
+        if (armsS[s]) mbar_wait_drain(FULL_S(s), (armsS[s] - 1) & 1, kDrainNs);
+    }
+    __syncwarp();
+  } else if (warp == BWDP_LOGIT_WARP || warp == BWDP_GRAD_WARP) {
+    // ------------------------------------------------------------ MMA
+    // Two issuing warps share the tensor pipe: one issues the logit MMAs of
+    // tile t+1 as soon as the row warps have read tile t's logits, the other
+    // the gradient MMAs of tile t once its G is stored, so that neither
+    // waits behind the other's barriers.  Each warp runs its loop converged
+    // (descriptor words stay warp-uniform); one elected lane issues.
+    const bool is_logit = warp == BWDP_LOGIT_WARP;
+    const uint32_t lead = elect_leader();
+    constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN64, 0, 0);
+    constexpr uint32_t IDESC_GX = idesc_bf16_f32(BM, D, 0, 1);    // A = G (K-major), B = X_s[J] (MN)
+    constexpr uint32_t IDESC_PT = idesc_bf16_f32(D, BN64, 1, 1);  // A = X_s[R]^T (MN), B = G (MN)
+    const uint32_t HI_1024 = sw128_desc_hi(1024);
+    const uint32_t dXtR_k[2] = {sw128_desc_lo(base + L::XT_R0, 16), sw128_desc_lo(base + L::XT_R1, 16)};
+    const uint32_t dXsR_k[2] = {sw128_desc_lo(base + L::XS_R0, 16), sw128_desc_lo(base + L::XS_R1, 16)};
+    const uint32_t dXsR_mn[2] = {sw128_desc_lo(base + L::XS_R0, L::BOX_I),
+                                 sw128_desc_lo(base + L::XS_R1, L::BOX_I)};
+    const uint32_t dXtJ_k0 = sw128_desc_lo(base + L::XT_J, 16);
+    const uint32_t dXsJ_k0 = sw128_desc_lo(base + L::XS_J, 16);
+    const uint32_t dXsJ_mn0 = sw128_desc_lo(base + L::XS_J, L::BOX_J);
+    const uint32_t dG_k = sw128_desc_lo(base + L::G, 16);
+    const uint32_t dG_mn = sw128_desc_lo(base + L::G, L::G_BYTES);
+    constexpr uint32_t J_STEP = L::TILE_J >> 4;
+    uint32_t nseq = 0, nJ = 0, nt = 0, np = 0;
+    bool ok = true, issued = false;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int m = item - (item / ipu) * ipu;
+      for (int w = 0; ok && w < 2; ++w) {
+        const int R0 = pair_seq_block(p, m, w);
+        if (R0 < 0) break;
+        const bool has1 = R0 + 1 < p.nblk;
+        const int nT0 = n_col_tiles64(p, R0);
+        const int nT = has1 ? n_col_tiles64(p, R0 + 1) : nT0;
+        if (!(ok = mbar_wait_warp(FULL_I, nseq & 1, wc, W_MMA_FULL_I))) break;
+        bool first_seq = true;
+        for (int J = 0; ok && J < nT; ++J) {
+          const int tt = nJ & 1, ts = nJ & 1;
+          for (int rs = 0; rs < 2; ++rs) {
+            if (rs == 0 && J >= nT0) continue;
+            if (rs == 1 && !has1) continue;
+            const bool first_p = rs == 0 || J >= nT0;
+            const bool last_p = rs == 1 || !has1;
+            if (is_logit) {
+              // Z_t, Z_s of tile (R, J) into the logit buffer
+              if (!(ok = mbar_wait_warp(FULL_T(tt), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+              if (!(ok = mbar_wait_warp(S_EMPTY, (nt & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
+              tc_fence_after();
+              const uint32_t xtj = dXtJ_k0 + tt * J_STEP, xsj = dXsJ_k0 + ts * J_STEP;
+              // K steps: 32 B within a 128 B row, then the next 64-column box
+#pragma unroll
+              for (int k = 0; k < D / 16; ++k)
+                umma_bf16_w_lead(lead, tmem + T_S, dXtR_k[rs] + (k >> 2) * (L::BOX_I >> 4) + (k & 3) * 2,
+                                 HI_1024, xtj + (k >> 2) * (L::BOX_J >> 4) + (k & 3) * 2, HI_1024,
+                                 IDESC_S, k > 0 ? 1u : 0u);
+              issued = true;
+              if (last_p) umma_commit_lead(lead, EMPTY_T(tt));
+              if (!(ok = mbar_wait_warp(FULL_S(ts), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+              tc_fence_after();
+#pragma unroll
+              for (int k = 0; k < D / 16; ++k)
+                umma_bf16_w_lead(lead, tmem + T_S + 64, dXsR_k[rs] + (k >> 2) * (L::BOX_I >> 4) + (k & 3) * 2,
+                                 HI_1024, xsj + (k >> 2) * (L::BOX_J >> 4) + (k & 3) * 2, HI_1024,
+                                 IDESC_S, k > 0 ? 1u : 0u);
+              umma_commit_lead(lead, S_FULL);
+            } else {
+              // dX_R += G X_s[J] and P^T (+)= X_s[R]^T G for tile (R, J).  G_FULL
+              // implies the tile's logits (hence its column tiles) are complete.
+              const int pb = np & 1;
+              if (!(ok = mbar_wait_warp(G_FULL, nt & 1, wc, W_MMA_G_FULL))) break;
+              if (first_p && !(ok = mbar_wait_warp(P_EMPTY(pb), ((np >> 1) & 1) ^ 1, wc, W_MMA_P_EMPTY)))
+                break;
+              if (first_seq && !(ok = mbar_wait_warp(DXI_EMPTY, (nseq & 1) ^ 1, wc, W_MMA_DXI_EMPTY)))
+                break;
+              first_seq = false;
+              tc_fence_after();
+              const uint32_t xsj = dXsJ_mn0 + ts * J_STEP;
+              // M = i, N = c, K = j (64); K steps of 32 B (G) and 2 KB (X_s[J])
+#pragma unroll
+              for (int k = 0; k < BN64 / 16; ++k)
+                umma_bf16_w_lead(lead, tmem + T_DX0 + rs * 128, dG_k + k * 2, HI_1024, xsj + k * 128,
+                                 HI_1024, IDESC_GX, (J > 0 || k > 0) ? 1u : 0u);
+              // M = c, N = j, K = i (128); K steps of 2 KB in both
+#pragma unroll
+              for (int k = 0; k < BM / 16; ++k)
+                umma_bf16_w_lead(lead, tmem + T_P + pb * 64, dXsR_mn[rs] + k * 128, HI_1024,
+                                 dG_mn + k * 128, HI_1024, IDESC_PT, (!first_p || k > 0) ? 1u : 0u);
+              issued = true;
+              umma_commit_lead(lead, G_EMPTY);
+              if (last_p) {
+                umma_commit_lead(lead, P_FULL(pb));
+                umma_commit_lead(lead, EMPTY_S(ts));
+                ++np;
+              }
+            }
+            ++nt;
+          }
+          ++nJ;
+        }
+        if (!ok) break;
+        if (!is_logit) {
+          umma_commit_lead(lead, EMPTY_I);
+          umma_commit_lead(lead, DXI_FULL);
+        }
+        ++nseq;
+      }
+    }
+    if (issued) {
+      const uint32_t drain = is_logit ? DRAIN_L : DRAIN_G;
+      umma_commit_lead(lead, drain);
+      mbar_wait_drain(drain, 0, kDrainNs);
+    }
+    __syncwarp();
+  } else if (warp >= BWD_EPI_WARP) {
+    // ------------------------------------------------------- epilogue
+    // Every f32 addition into dX goes out as a TMA reduce-add of a 32 x 32
+    // box staged in this warp's 4 KB of shared memory (128-byte swizzle).
+    // P^T lane c = 32q + lane holds dX[J*64 + j][c] for the tile's 64 columns
+    // j, so it is staged transposed: one 128-byte row of the box per j.
+    const int q = warp - BWD_EPI_WARP;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t stg = base + L::STG + q * L::STG_BYTES;
+    uint32_t np = 0, nseq = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int u = item / ipu, m = item - u * ipu;
+      const Unit U = decode_unit(p, u);
+      for (int w = 0; ok && w < 2; ++w) {
+        const int R0 = pair_seq_block(p, m, w);
+        if (R0 < 0) break;
+        const bool has1 = R0 + 1 < p.nblk;
+        const int nT = n_col_tiles64(p, has1 ? R0 + 1 : R0);
+        for (int J = 0; J < nT; ++J) {
+          const int b = np & 1;
+          ok = mbar_wait(P_FULL(b), (np >> 1) & 1, wc, W_EPI_P_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int jb = 0; jb < 2; ++jb) {
+            float v[32];
+            tmem_ld32(tmem + lane_addr + T_P + b * 64 + jb * 32, v);
+            tmem_wait_ld();
+            if (jb == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(P_EMPTY(b));
+            }
+            if (lane == 0) bulk_wait_read<0>();   // the previous box has left the buffer
+            __syncwarp();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              st_shared_b32(stg + jj * 128 + (((lane >> 2) ^ (jj & 7)) << 4) + (lane & 3) * 4, v[jj]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int row0 = J * BN64 + jb * 32;
+            if (lane == 0) {
+              if (row0 < p.N) tma_reduce_add_4d(&U.seg->tm_dx, stg, q * 32, row0, U.h, U.b);
+              bulk_commit();
+            }
+          }
+          ++np;
+        }
+        if (!ok) break;
+        // dX rows of the pair: lane = row, 32-column boxes
+        ok = mbar_wait(DXI_FULL, nseq & 1, wc, W_EPI_DXI_FULL);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        for (int rs = 0; rs < 2; ++rs) {
+          const int row0 = (R0 + rs) * BM + q * 32;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tmem_ld32(tmem + lane_addr + T_DX0 + rs * 128 + c * 32, v);
+            tmem_wait_ld();
+            if (rs == 1 && c == D / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(DXI_EMPTY);
+            }
+            if (rs == 1 && !has1) continue;
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+            const uint32_t rowp = stg + lane * 128;
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4)
+              st_shared_v4(rowp + ((k4 ^ (lane & 7)) << 4), __float_as_uint(v[4 * k4]),
+                           __float_as_uint(v[4 * k4 + 1]), __float_as_uint(v[4 * k4 + 2]),
+                           __float_as_uint(v[4 * k4 + 3]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (row0 < p.N) tma_reduce_add_4d(&U.seg->tm_dx, stg, c * 32, row0, U.h, U.b);
+              bulk_commit();
+            }
+          }
+        }
+        ++nseq;
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  } else {
+    // --------------------------------------------------- row warpgroups
+    const int q = warp & 3;
+    const int wg = warp >> 2;      // 16-column slice of each 64-column tile
+    const int r = q * 32 + lane;
+    const float sl2 = p.sl2;
+    const uint32_t gsm = base + L::G + r * 128;  // row r of G: 128 bytes, chunks 2wg, 2wg+1
+    uint32_t nt = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      const int u = item / ipu, m = item - u * ipu;
+      const Unit U = decode_unit(p, u);
+      for (int w = 0; ok && w < 2; ++w) {
+        const int R0 = pair_seq_block(p, m, w);
+        if (R0 < 0) break;
+        const bool has1 = R0 + 1 < p.nblk;
+        const int nT0 = n_col_tiles64(p, R0);
+        const int nT = has1 ? n_col_tiles64(p, R0 + 1) : nT0;
+        // per-row constants of both row blocks
+        float bt[2], bs[2], mul[2];
+        int lim[2];
+#pragma unroll
+        for (int rs = 0; rs < 2; ++rs) {
+          const int row = (R0 + rs) * BM + r;
+          const bool rvalid = row < p.N && (rs == 0 || has1);
+          bt[rs] = bs[rs] = mul[rs] = 0.f;
+          if (rvalid) {
+            const float4 st4 = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + row];
+            bt[rs] = -st4.y * kLog2e;
+            bs[rs] = -st4.z * kLog2e;
+            const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(p.N);
+            mul[rs] = up * p.scale;   // the logit scale of dX_s is folded into G
+          }
+          lim[rs] = !rvalid ? -1 : (p.causal ? min(row, p.N - 1) : p.N - 1);
+        }
+        const float2 sl2v = make_float2(sl2, sl2), m1 = make_float2(-1.f, -1.f);
+        for (int J = 0; ok && J < nT; ++J) {
+          for (int rs = 0; rs < 2; ++rs) {
+            if (rs == 0 && J >= nT0) continue;
+            if (rs == 1 && !has1) continue;
+            ok = mbar_wait(S_FULL, nt & 1, wc, W_SM_S_FULL);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + T_S + wg * 16;
+            float t[16], s[16];
+            tmem_ld16(ta, t);
+            tmem_ld16(ta + 64, s);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(S_EMPTY);
+            const float btr = rs ? bt[1] : bt[0], bsr = rs ? bs[1] : bs[0];
+            const float mr = rs ? mul[1] : mul[0];
+            const int limr = rs ? lim[1] : lim[0];
+            const float2 btv = make_float2(btr, btr), bsv = make_float2(bsr, bsr),
+                         mulv = make_float2(mr, mr);
+            const int col0 = J * BN64 + wg * 16;
+            const bool need_mask = col0 + 15 > limr;
+            uint32_t pk[8];
+#pragma unroll
+            for (int k = 0; k < 16; k += 2) {
+              const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
+              const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
+              const float2 et = ex2_approx2(at), es = ex2_approx2(as);
+              float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
+              if (need_mask) {
+                g.x = (col0 + k <= limr) ? g.x : 0.f;
+                g.y = (col0 + k + 1 <= limr) ? g.y : 0.f;
+              }
+              pk[k >> 1] = pack_bf16x2(g.x, g.y);
+            }
+            // the previous tile's gradient MMAs have read G
+            ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int cc = 2 * wg + h2;  // 16-byte chunk within the 128-byte row
+              st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[4 * h2], pk[4 * h2 + 1], pk[4 * h2 + 2],
+                           pk[4 * h2 + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(G_FULL);
+            ++nt;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == BWDP_LOGIT_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ------------------------------------------------------------ launchers
 template <int D>
 static cudaError_t launch_fwd(const TcParams& p, int grid, cudaStream_t stream) {
@@ -1281,17 +1766,26 @@ cudaError_t tc_launch_fwd(const TcParams& p, int d, int grid, cudaStream_t strea
 
 cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t stream) {
   if (d == 64) return launch_bwd<64>(p, grid, stream);
-  cudaError_t e = cudaFuncSetAttribute(relkl_bwd_tc64_kernel,
+  if (p.nblk <= kPairMinBlocks - 1) {
+    cudaError_t e = cudaFuncSetAttribute(relkl_bwd_tc64_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Bwd64Smem::ALLOC);
+    if (e != cudaSuccess) return e;
+    relkl_bwd_tc64_kernel<<<grid, BWD_THREADS, Bwd64Smem::ALLOC, stream>>>(p);
+    return cudaGetLastError();
+  }
+  // work items of the pair kernel: ceil(npb / 2) per unit, npb = ceil(nblk / 2)
+  TcParams q = p;
+  const int units = p.n_items / p.n_pairs;
+  q.n_pairs = ((p.nblk + 1) / 2 + 1) / 2;
+  q.n_items = units * q.n_pairs;
+  cudaError_t e = cudaFuncSetAttribute(relkl_bwd_pair_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Bwd64Smem::ALLOC);
+                                       BwdPairSmem::ALLOC);
   if (e != cudaSuccess) return e;
-  relkl_bwd_tc64_kernel<<<grid, BWD_THREADS, Bwd64Smem::ALLOC, stream>>>(p);
+  relkl_bwd_pair_kernel<<<grid, BWDP_THREADS, BwdPairSmem::ALLOC, stream>>>(q);
   return cudaGetLastError();
 }
 
-size_t tc_smem_bytes(int d, int is_bwd) {
-  if (is_bwd) return d == 64 ? BwdSmem<64>::ALLOC : Bwd64Smem::ALLOC;
-  return d == 64 ? FwdSmem<64>::ALLOC : FwdSmem<128>::ALLOC;
-}
 
 }  // namespace relkl

@@ -51,6 +51,14 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def bwd_kernel_name(w) -> str:
+    """The backward kernel the library launches for this workload (tcgen05 path)."""
+    if w.d == 64:
+        return "relkl_bwd_tc_kernel"
+    # 128-row blocks: more than 32 of them take the kernel that pairs adjacent blocks
+    return "relkl_bwd_pair_kernel" if (w.N + 127) // 128 > 32 else "relkl_bwd_tc64_kernel"
+
+
 def traffic_record(kernel: str):
     """Per-launch DRAM bytes from the committed ncu summary, if it matches the current kernel source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -383,7 +391,8 @@ def main():
     bwd_avg = sum(bwd_ms) / len(bwd_ms)
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
     achieved = fl_bwd / (bwd_avg * 1e-3) / 1e12
-    traffic = traffic_record("relkl_bwd_tc64_kernel" if w.d == 128 else "relkl_bwd_tc_kernel")
+    bwd_kernel = bwd_kernel_name(w)
+    traffic = traffic_record(bwd_kernel)
 
     result = None
     if rank == 0:
@@ -404,7 +413,7 @@ def main():
             "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
             "fwd_tflops": fl_fwd / (fwd_avg * 1e-3) / 1e12,
             "bwd_tflops": fl_bwd / (bwd_avg * 1e-3) / 1e12,
-            "roofline": {"kernel": "relkl_bwd_tc64_kernel" if w.d == 128 else "relkl_bwd_tc_kernel",
+            "roofline": {"kernel": bwd_kernel,
                          "bound": "tensor", "achieved": achieved,
                          "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
                          "traffic": traffic,

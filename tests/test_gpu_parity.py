@@ -66,6 +66,27 @@ def test_tc_shapes_rope_pi(N, d, causal, B, H):
     check_full(xt, xs, causal=causal, path=1)
 
 
+# N > 4096 takes the backward that pairs adjacent 128-row blocks: odd block
+# counts (a last pair with one block), ragged tails, both masks.
+@pytest.mark.parametrize("N,causal,B,H", [
+    (4200, True, 1, 2), (4352, False, 1, 1), (4097, True, 2, 1), (4480, True, 1, 1),
+])
+def test_tc_paired_row_blocks(N, causal, B, H):
+    xt, xs = q_inputs(B, H, N, 128, seed=N, causal=causal)
+    check_full(xt, xs, causal=causal, path=1)
+
+
+def test_tc_paired_row_blocks_upstream_gradient_and_zero():
+    xt, xs = q_inputs(1, 1, 4300, 128, seed=31)
+    dkl = torch.randn(1, 1, 4300, generator=torch.Generator().manual_seed(3)) / 4300
+    check_full(xt, xs, dkl=dkl)
+    g = xt.cuda()
+    kl, st = rk.relkl_fwd(g, g.clone())
+    dx = rk.relkl_bwd(g, g.clone(), st)
+    torch.cuda.synchronize()
+    assert torch.all(kl == 0) and torch.all(dx == 0)
+
+
 def test_tc_value_relation_small_kl():
     # V-like: student = teacher + small noise, KL ~ 1e-3 per row
     xt, xs = workload.gaussian_pair((1, 2, 640, 128), seed=5, noise=0.05, dtype=torch.bfloat16)
@@ -130,6 +151,22 @@ def test_fused_qkv_gqa_small():
         ref = dense.fwd(*x[r])
         assert_kl(to_np(kl), ref["kl"], what=f"kl[{r}]")
         assert_stats(to_np(st), ref)
+        assert_dx(to_np(dx), dense.bwd(*x[r]), DX_TOL_BF16)
+
+
+def test_fused_qkv_gqa_paired_blocks():
+    g = workload.Workload("gqa_paired", B=1, H=2, H_kv=1, N=4200, d=128, dtype="bf16", causal=True,
+                          relations=("q", "k", "v"), rope_base=5e5, pi_factor=4.0, v_noise=0.05,
+                          seed=23)
+    x = workload.generate(g)
+    pairs = [(x[r][0].cuda(), x[r][1].cuda()) for r in "qkv"]
+    outs = rk.relkl_fwd_qkv(pairs)
+    dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs])
+    torch.cuda.synchronize()
+    _device_ok()
+    for r, (kl, st), dx in zip("qkv", outs, dxs):
+        ref = dense.fwd(*x[r])
+        assert_kl(to_np(kl), ref["kl"], what=f"kl[{r}]")
         assert_dx(to_np(dx), dense.bwd(*x[r]), DX_TOL_BF16)
 
 
