@@ -48,3 +48,23 @@ def test_v_noise_level():
                           relations=("v",), rope_base=1e4, pi_factor=8.0, v_noise=0.1, seed=2)
     vt, vs = workload.generate(w)["v"]
     assert abs(float((vs - vt).std()) - 0.1) < 0.005
+
+
+def test_chain_workload_shapes_determinism_and_projection():
+    cw = workload.CHAIN_CONFIGS["chain_small"]
+    a, b = workload.generate_chain(cw), workload.generate_chain(cw)
+    assert torch.equal(a["h_s"], b["h_s"]) and torch.equal(a["x"]["k"][1], b["x"]["k"][1])
+    assert a["h_t"].shape == (cw.B, cw.N, cw.D) and a["h_t"].dtype == torch.bfloat16
+    assert a["w"]["q"].shape == (cw.D, cw.H * cw.d) and a["w"]["v"].shape == (cw.D, cw.H_kv * cw.d)
+    for rel in "qkv":
+        xt, xs = a["x"][rel]
+        assert xt.shape == (cw.B, cw.heads(rel), cw.N, cw.d) and xt.is_contiguous()
+    # V is the plain projection of the rounded hidden states; K is its rotation at p / s
+    hv = (a["h_s"].float() @ a["w"]["v"].float()).reshape(cw.B, cw.N, cw.H_kv, cw.d).permute(0, 2, 1, 3)
+    assert torch.equal(a["x"]["v"][1], hv.to(torch.bfloat16))
+    hk = (a["h_s"].float() @ a["w"]["k"].float()).reshape(cw.B, cw.N, cw.H_kv, cw.d).permute(0, 2, 1, 3)
+    rk = workload.rope_rotate(hk, a["pos_s"], cw.rope_base).to(torch.bfloat16)
+    assert torch.equal(a["x"]["k"][1], rk)
+    # student hidden states differ from the teacher's by the configured noise
+    diff = (a["h_s"].float() - a["h_t"].float()).std().item()
+    assert 0.08 < diff < 0.12
