@@ -20,13 +20,19 @@ RELKL_FP32 = 1
 EXPORTS = ("relkl_workspace_bytes", "relkl_workspace_init", "relkl_fwd", "relkl_bwd",
            "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_get_device_error",
            "relkl_set_wait_timeout_ns", "relkl_status_string", "relkl_last_cuda_error",
-           "relkl_path_for", "relkl_fwd_noalloc")
+           "relkl_path_for", "relkl_fwd_noalloc", "relkl_rope_bwd", "relkl_weight_grad")
 
 
 class relkl_desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("stride", ctypes.c_int64 * 4), ("dtype", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("reserved", ctypes.c_int32)]
+
+
+class relkl_rope(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_double), ("pos_scale", ctypes.c_double),
+                ("pos_offset", ctypes.c_double), ("apply", ctypes.c_int32),
                 ("reserved", ctypes.c_int32)]
 
 
@@ -64,6 +70,11 @@ def _declare(lib):
     lib.relkl_path_for.argtypes = [ctypes.POINTER(relkl_desc)]
     lib.relkl_fwd_noalloc.restype = ctypes.c_int
     lib.relkl_fwd_noalloc.argtypes = [ctypes.POINTER(relkl_desc), _vp, _vp, _vp, _vp, _vp]
+    i32 = ctypes.c_int32
+    lib.relkl_rope_bwd.restype = ctypes.c_int
+    lib.relkl_rope_bwd.argtypes = [i32, i32, i32, i32, _vp, ctypes.POINTER(relkl_rope), i32, _vp, _vp]
+    lib.relkl_weight_grad.restype = ctypes.c_int
+    lib.relkl_weight_grad.argtypes = [ctypes.c_int64, i32, i32, _vp, _vp, _vp, _vp]
     return lib
 
 
@@ -85,7 +96,7 @@ class RelklError(RuntimeError):
     def __init__(self, code: int, where: str):
         msg = lib().relkl_status_string(code).decode()
         if code == RELKL_ERR_CUDA:
-            msg += f" (cudaError {lib().relkl_last_cuda_error()})"
+            msg += f" (CUDA / cuBLAS status {lib().relkl_last_cuda_error()})"
         super().__init__(f"{where}: {msg}")
         self.code = code
 

@@ -21,6 +21,11 @@ cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t strea
 cudaError_t simt_launch_fwd(const SimtParams& p, cudaStream_t stream);
 cudaError_t simt_launch_bwd(const SimtParams& p, cudaStream_t stream);
 cudaError_t launch_zero(float* ptr, int64_t n, int num_sms, cudaStream_t stream);
+cudaError_t launch_rope_bwd(const float* dx, void* out, int B, int H, int N, int d, bool bf16_out,
+                            double base, double pos_scale, double pos_offset, int apply,
+                            cudaStream_t stream);
+int chain_weight_grad(long long rows, int D, int cols, const void* h, const void* dx_pre,
+                      float* dw, cudaStream_t stream);
 }  // namespace relkl
 
 using namespace relkl;
@@ -424,6 +429,40 @@ const char* relkl_status_string(relkl_status s) {
 }
 
 int32_t relkl_last_cuda_error(void) { return g_last_cuda; }
+
+relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const float* dx_post,
+                            const relkl_rope* rope, int32_t out_dtype, void* dx_pre,
+                            void* stream) {
+  if (!rope || B < 0 || H < 0 || N < 0 || d < 2 || d > 512 || (d & 1)) return RELKL_ERR_INVALID;
+  if (out_dtype != RELKL_BF16 && out_dtype != RELKL_FP32) return RELKL_ERR_INVALID;
+  if (rope->reserved != 0 || (rope->apply != 0 && rope->apply != 1)) return RELKL_ERR_INVALID;
+  if (!std::isfinite(rope->base) || !(rope->base > 1.0) || !std::isfinite(rope->pos_scale) ||
+      !std::isfinite(rope->pos_offset))
+    return RELKL_ERR_INVALID;
+  const long long tokens = static_cast<long long>(B) * N;
+  if (tokens == 0 || H == 0) return RELKL_OK;
+  if (tokens > 0x7fffffffLL) return RELKL_ERR_INVALID;
+  if (!dx_post || !dx_pre || !aligned(dx_post, 4) || !aligned(dx_pre, out_dtype == RELKL_BF16 ? 2 : 4))
+    return RELKL_ERR_INVALID;
+  cudaError_t e = launch_rope_bwd(dx_post, dx_pre, B, H, N, d, out_dtype == RELKL_BF16, rope->base,
+                                  rope->pos_scale, rope->pos_offset, rope->apply,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
+}
+
+relkl_status relkl_weight_grad(int64_t rows, int32_t D, int32_t cols, const void* h,
+                               const void* dx_pre, float* dw, void* stream) {
+  if (rows < 1 || rows > 0x7fffffffLL || D < 1 || cols < 1 || (D % 8) || (cols % 8))
+    return RELKL_ERR_INVALID;
+  if (!h || !dx_pre || !dw || !aligned(h, 16) || !aligned(dx_pre, 16) || !aligned(dw, 16))
+    return RELKL_ERR_INVALID;
+  const int st = chain_weight_grad(rows, D, cols, h, dx_pre, dw, static_cast<cudaStream_t>(stream));
+  if (st != 0) {
+    g_last_cuda = st;
+    return RELKL_ERR_CUDA;
+  }
+  return RELKL_OK;
+}
 
 }  // extern "C"
 

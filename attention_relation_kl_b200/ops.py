@@ -22,7 +22,7 @@ from ._abi import check, relkl_desc
 __all__ = ["relkl_fwd", "relkl_bwd", "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_workspace_bytes",
            "relkl_workspace_init", "relkl_get_device_error", "relkl_set_wait_timeout_ns",
            "relkl_path_for", "workspace", "make_desc", "relation_kl", "RelationKL",
-           "relkl_fwd_noalloc"]
+           "relkl_fwd_noalloc", "relkl_rope_bwd", "relkl_weight_grad", "student_weight_grads"]
 
 _DTYPES = {torch.bfloat16: _abi.RELKL_BF16, torch.float32: _abi.RELKL_FP32}
 
@@ -238,3 +238,64 @@ def relation_kl(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,
                 scale: float = 0.0) -> torch.Tensor:
     """Differentiable per-row KL(R_t || R_s) of one relation, shape [B, H, N]."""
     return RelationKL.apply(x_t, x_s, causal, scale)
+
+
+# ------------------------------------------------ chain rule to the weights
+
+def relkl_rope_bwd(dx_post: torch.Tensor, base: float, pos_scale: float = 1.0,
+                   pos_offset: float = 0.0, apply: bool = True,
+                   out_dtype: torch.dtype = torch.bfloat16, *,
+                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """RoPE backward plus head/token transpose: [B, H, N, d] fp32 -> [B, N, H, d]."""
+    _cuda(dx_post, "dx_post")
+    if dx_post.dtype != torch.float32 or dx_post.dim() != 4 or not dx_post.is_contiguous():
+        raise ValueError("dx_post must be a contiguous float32 [B, H, N, d] tensor")
+    if out_dtype not in _DTYPES:
+        raise TypeError(f"unsupported output dtype {out_dtype}")
+    B, H, N, d = (int(v) for v in dx_post.shape)
+    if out is None:
+        out = torch.empty(B, N, H, d, dtype=out_dtype, device=dx_post.device)
+    rope = _abi.relkl_rope(float(base), float(pos_scale), float(pos_offset), 1 if apply else 0, 0)
+    check(_abi.lib().relkl_rope_bwd(B, H, N, d, _ptr(dx_post), ctypes.byref(rope),
+                                    _DTYPES[out_dtype], _ptr(out), _stream(dx_post.device, stream)),
+          "relkl_rope_bwd")
+    return out
+
+
+def relkl_weight_grad(h: torch.Tensor, dx_pre: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """dW [D, cols] fp32 = h^T dx_pre over token rows (h [..., D], dx_pre [..., cols], bf16)."""
+    _cuda(h, "h")
+    _cuda(dx_pre, "dx_pre")
+    if h.dtype != torch.bfloat16 or dx_pre.dtype != torch.bfloat16:
+        raise TypeError("h and dx_pre must be bfloat16")
+    if not h.is_contiguous() or not dx_pre.is_contiguous():
+        raise ValueError("h and dx_pre must be contiguous")
+    D = int(h.shape[-1])
+    rows = h.numel() // D
+    cols = dx_pre.numel() // rows if rows else 0
+    if rows * cols != dx_pre.numel():
+        raise ValueError("h and dx_pre disagree on the number of token rows")
+    if out is None:
+        out = torch.empty(D, cols, dtype=torch.float32, device=h.device)
+    check(_abi.lib().relkl_weight_grad(rows, D, cols, _ptr(h), _ptr(dx_pre), _ptr(out),
+                                       _stream(h.device, stream)), "relkl_weight_grad")
+    return out
+
+
+def student_weight_grads(pairs: Dict[str, Tuple[torch.Tensor, torch.Tensor]], h_s: torch.Tensor,
+                         rope_base: float, pos_scale: float, causal: bool = True,
+                         dkl: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
+    """dW_q, dW_k, dW_v of the student: relation-KL forward and backward over the
+    relations given ({rel: (x_t, x_s)}, one fused launch each), RoPE backward for q
+    and k at the student's positions, and the weight gradient against h_s [B, N, D]."""
+    rels = list(pairs)
+    outs = relkl_fwd_qkv([pairs[r] for r in rels], causal)
+    dxs = relkl_bwd_qkv([pairs[r] for r in rels], [o[1] for o in outs],
+                        None if dkl is None else [dkl.get(r) for r in rels], causal)
+    grads = {}
+    for r, dx in zip(rels, dxs):
+        pre = relkl_rope_bwd(dx, rope_base, pos_scale, 0.0, apply=(r != "v"))
+        grads[r] = relkl_weight_grad(h_s, pre)
+    return grads
+

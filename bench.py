@@ -257,6 +257,79 @@ def run_sweep(args):
     return 0
 
 
+# ------------------------------------------- chain rule to the weights (one GPU)
+
+def run_chain(args):
+    """Time the steps from dX_s to dW_q, dW_k, dW_v at the LLaMA2-7B layer shape
+    (D = 4096, 32 heads of 128) and N = 32768: the RoPE backward with the
+    head/token transpose (HBM-bound: reads dX_s fp32, writes bf16) and the
+    three weight-gradient GEMMs (2 * rows * D * cols flops each).  One JSON line.
+    """
+    import attention_relation_kl_b200 as rk
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cw = workload.CHAIN_CONFIGS["chain_llama2_n32k"]
+    c = workload.generate_chain(cw)
+    rels = ("q", "k", "v")
+    pairs = [(c["x"][r][0].to(dev), c["x"][r][1].to(dev)) for r in rels]
+    hs = c["h_s"].to(dev)
+    del c
+    ws = rk.workspace(dev)
+    outs = rk.relkl_fwd_qkv(pairs, cw.causal, ws=ws)
+    dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, cw.causal, ws=ws)
+    pres = [torch.empty(cw.B, cw.N, cw.heads(r), cw.d, dtype=torch.bfloat16, device=dev)
+            for r in rels]
+    dws = [torch.empty(cw.D, cw.heads(r) * cw.d, dtype=torch.float32, device=dev) for r in rels]
+    scale = 1.0 / cw.pi_factor
+
+    def rope_all():
+        for r, dx, pre in zip(rels, dxs, pres):
+            rk.relkl_rope_bwd(dx, cw.rope_base, scale, 0.0, r != "v", torch.bfloat16, out=pre)
+
+    def gemm_all():
+        for pre, dw in zip(pres, dws):
+            rk.relkl_weight_grad(hs, pre, out=dw)
+
+    for _ in range(max(3, args.warmup)):
+        rope_all()
+        gemm_all()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    steps = max(1, args.steps)
+    rope_ms = gemm_ms = bwd_ms = 0.0
+    for _ in range(steps):
+        ev[0].record()
+        rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, cw.causal, out=dxs, ws=ws)
+        ev[1].record()
+        rope_all()
+        ev[2].record()
+        gemm_all()
+        ev[3].record()
+        torch.cuda.synchronize()
+        bwd_ms += ev[0].elapsed_time(ev[1]) / steps
+        rope_ms += ev[1].elapsed_time(ev[2]) / steps
+        gemm_ms += ev[2].elapsed_time(ev[3]) / steps
+    peaks, src = load_peaks()
+    elems = sum(dx.numel() for dx in dxs)
+    rope_bytes = elems * (4 + 2)
+    rows = cw.B * cw.N
+    gemm_fl = sum(2.0 * rows * cw.D * cw.heads(r) * cw.d for r in rels)
+    print(json.dumps({
+        "chain": cw.name, "B": cw.B, "N": cw.N, "D": cw.D, "H": cw.H, "H_kv": cw.H_kv, "d": cw.d,
+        "steps": steps,
+        "rope_bwd_ms": rope_ms, "rope_bwd_gbs": rope_bytes / (rope_ms * 1e-3) / 1e9,
+        "rope_bwd_frac_hbm": rope_bytes / (rope_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "rope_bwd_bytes": rope_bytes,
+        "weight_grad_ms": gemm_ms, "weight_grad_tflops": gemm_fl / (gemm_ms * 1e-3) / 1e12,
+        "weight_grad_frac_bf16": gemm_fl / (gemm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "weight_grad_flops": gemm_fl,
+        "relation_bwd_ms": bwd_ms,
+        "chain_share_of_bwd": (rope_ms + gemm_ms) / bwd_ms,
+        "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"], "source": src},
+    }), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def main():
@@ -272,6 +345,9 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="sequence-length sweep (B*N = 65536): one JSON line per N with "
                          "throughput and peak extra memory, instead of the bench line")
+    ap.add_argument("--chain", action="store_true",
+                    help="time the chain rule to the Q/K/V weights (RoPE backward, weight "
+                         "gradient GEMMs) at the LLaMA2-7B layer shape, N = 32768")
     args = ap.parse_args()
     w = workload.get_config(args.config)
 
@@ -279,6 +355,8 @@ def main():
         return run_reference(args, w)
     if args.sweep:
         return run_sweep(args)
+    if args.chain:
+        return run_chain(args)
 
     import torch.distributed as dist
     import attention_relation_kl_b200 as rk

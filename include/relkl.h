@@ -170,6 +170,63 @@ int32_t relkl_path_for(const relkl_desc* desc);
 relkl_status relkl_fwd_noalloc(const relkl_desc* desc, const void* x_t, const void* x_s,
                                float* kl, float* stats, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Chain rule from dX_s to the student's projection weights.
+ *
+ * LinearARD trains only the student's Q/K/V projections (pith.science
+ * verdict page, pith_extraction.minor_comments); the student's relation
+ * inputs are X_s = RoPE_s(H_s W_x) for x in {q, k} and X_s = H_s W_v for V,
+ * with H_s [B, N, D] the student's hidden states and the heads of X laid side
+ * by side per token.  The pages stop at the logit gradient; the two steps
+ * below are the plain chain rule applied to relkl_bwd's dX_s.
+ */
+
+/* Rotate-half RoPE (RoFormer's rotary embedding in LLaMA's pairing): pair
+ * (i, i + d/2) of token n rotates by pos(n) * base^(-2i/d), with
+ * pos(n) = pos_offset + n * pos_scale (pos_scale = 1/s for positional
+ * interpolation by s).                                                       */
+typedef struct {
+  double base;        /* > 1, e.g. 10000 */
+  double pos_scale;   /* finite */
+  double pos_offset;  /* finite */
+  int32_t apply;      /* 1: the input carried RoPE (Q, K); 0: it did not (V) */
+  int32_t reserved;   /* must be 0 */
+} relkl_rope;
+
+/* RoPE backward with the head/token transpose the weight gradient needs.
+ *
+ *   dx_pre[b, n, h, :] = R(pos(n))^T dx_post[b, h, n, :]
+ *
+ * where R is the rotation above (the identity when rope->apply == 0): for
+ * each pair, (g_a, g_b) -> (g_a cos + g_b sin, g_b cos - g_a sin).  Angles are
+ * formed in double precision, the rotation in float32.
+ *   dx_post  : float [B, H, N, d] contiguous (relkl_bwd's dx_s), in.
+ *   dx_pre   : [B, N, H, d] contiguous, out, overwritten; element type
+ *              out_dtype (RELKL_BF16 to feed relkl_weight_grad, or RELKL_FP32).
+ * d must be even and 2 <= d <= 512; B, H, N >= 0 (zero work is a no-op).
+ * RELKL_ERR_INVALID for bad shapes, null pointers with work to do, a
+ * non-finite or non-positive base, non-finite positions or reserved != 0.    */
+relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const float* dx_post,
+                            const relkl_rope* rope, int32_t out_dtype, void* dx_pre,
+                            void* stream);
+
+/* Weight gradient over the token rows:
+ *
+ *   dw[D, cols] = h[rows, D]^T dx_pre[rows, cols]
+ *
+ * (rows = B*N tokens, cols = heads * d), overwriting dw.  One dense GEMM on
+ * the tensor cores through cuBLAS: bf16 operands, float32 accumulation and
+ * result.  The library keeps one cuBLAS handle per device, created on the
+ * first call without a workspace; calls are serialised on it.
+ *   h      : bf16 [rows, D] row-major (the student's hidden states), in.
+ *   dx_pre : bf16 [rows, cols] row-major (relkl_rope_bwd's output), in.
+ *   dw     : float [D, cols] row-major, out.
+ * 1 <= rows <= 2^31 - 1, D >= 1, cols >= 1; pointers 16-byte aligned and
+ * D, cols multiples of 8.  RELKL_ERR_INVALID otherwise; RELKL_ERR_CUDA with
+ * the cuBLAS status in relkl_last_cuda_error() when cuBLAS fails.            */
+relkl_status relkl_weight_grad(int64_t rows, int32_t D, int32_t cols, const void* h,
+                               const void* dx_pre, float* dw, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -118,3 +118,47 @@ def test_wait_timeout_setting_roundtrip():
     lib = _abi.lib()
     old = lib.relkl_set_wait_timeout_ns(12345)
     assert lib.relkl_set_wait_timeout_ns(old) == 12345
+
+
+def _rope(base=1e4, scale=0.25, offset=0.0, apply=1, reserved=0):
+    return _abi.relkl_rope(base, scale, offset, apply, reserved)
+
+
+def test_rope_bwd_validation():
+    lib = _abi.lib()
+    buf = ctypes.c_void_p(4096)   # never dereferenced: every case fails validation or is empty
+    good = _rope()
+    inv = _abi.RELKL_ERR_INVALID
+    cases = [
+        (1, 2, 8, 7, buf, good, _abi.RELKL_BF16, buf),          # odd d
+        (1, 2, 8, 0, buf, good, _abi.RELKL_BF16, buf),          # d < 2
+        (1, 2, 8, 514, buf, good, _abi.RELKL_BF16, buf),        # d > 512
+        (-1, 2, 8, 64, buf, good, _abi.RELKL_BF16, buf),        # negative B
+        (1, 2, 8, 64, buf, good, 7, buf),                       # unknown dtype
+        (1, 2, 8, 64, None, good, _abi.RELKL_BF16, buf),        # null input with work
+        (1, 2, 8, 64, buf, good, _abi.RELKL_BF16, None),        # null output with work
+        (1, 2, 8, 64, buf, _rope(base=1.0), _abi.RELKL_BF16, buf),
+        (1, 2, 8, 64, buf, _rope(base=float("nan")), _abi.RELKL_BF16, buf),
+        (1, 2, 8, 64, buf, _rope(scale=float("inf")), _abi.RELKL_BF16, buf),
+        (1, 2, 8, 64, buf, _rope(apply=2), _abi.RELKL_BF16, buf),
+        (1, 2, 8, 64, buf, _rope(reserved=1), _abi.RELKL_BF16, buf),
+        (1, 2, 8, 64, ctypes.c_void_p(4097), good, _abi.RELKL_FP32, buf),   # misaligned input
+    ]
+    for B, H, N, d, src, rope, dt, dst in cases:
+        assert lib.relkl_rope_bwd(B, H, N, d, src, ctypes.byref(rope), dt, dst, None) == inv
+    assert lib.relkl_rope_bwd(1, 2, 8, 64, buf, None, _abi.RELKL_BF16, buf, None) == inv
+    # zero work: nothing to check, nothing enqueued
+    assert lib.relkl_rope_bwd(0, 2, 8, 64, None, ctypes.byref(good), _abi.RELKL_BF16, None, None) == 0
+    assert lib.relkl_rope_bwd(1, 0, 8, 64, None, ctypes.byref(good), _abi.RELKL_BF16, None, None) == 0
+
+
+def test_weight_grad_validation():
+    lib = _abi.lib()
+    p = ctypes.c_void_p(4096)
+    inv = _abi.RELKL_ERR_INVALID
+    for rows, D, cols, h, dx, dw in [
+        (0, 64, 64, p, p, p), (8, 0, 64, p, p, p), (8, 64, 0, p, p, p), (8, 60, 64, p, p, p),
+        (8, 64, 12, p, p, p), (2 ** 31, 64, 64, p, p, p), (8, 64, 64, None, p, p),
+        (8, 64, 64, p, None, p), (8, 64, 64, p, p, None), (8, 64, 64, ctypes.c_void_p(4104), p, p),
+    ]:
+        assert lib.relkl_weight_grad(rows, D, cols, h, dx, dw, None) == inv
