@@ -51,8 +51,14 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+# fp32 CUDA-core path: 148 SMs x 128 fp32 lanes x 2 flops (FMA) x 1.965 GHz
+FP32_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def bwd_kernel_name(w) -> str:
-    """The backward kernel the library launches for this workload (tcgen05 path)."""
+    """The backward kernel the library launches for this workload."""
+    if w.dtype != "bf16" or w.d not in (64, 128):
+        return "relkl_bwd_simt_kernel"
     if w.d == 64:
         return "relkl_bwd_tc_kernel"
     # 128-row blocks: more than 32 of them take the kernel that pairs adjacent blocks
@@ -465,7 +471,9 @@ def main():
     tokens = w.B * w.N * world / (ms_step * 1e-3)
 
     peaks, peak_src = load_peaks()
+    tensor_path = w.dtype == "bf16" and w.d in (64, 128)
     peak_tf = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    roof_peak = peak_tf if tensor_path else FP32_CORE_TFLOPS
     bwd_avg = sum(bwd_ms) / len(bwd_ms)
     fwd_avg = sum(fwd_ms) / len(fwd_ms)
     achieved = fl_bwd / (bwd_avg * 1e-3) / 1e12
@@ -481,7 +489,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
                        "relations": "".join(w.relations), "causal": w.causal,
                        "parallelism": f"replicas{world}" if world > 1 else "single",
@@ -492,10 +500,12 @@ def main():
             "fwd_tflops": fl_fwd / (fwd_avg * 1e-3) / 1e12,
             "bwd_tflops": fl_bwd / (bwd_avg * 1e-3) / 1e12,
             "roofline": {"kernel": bwd_kernel,
-                         "bound": "tensor", "achieved": achieved,
-                         "peak": peak_tf, "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                         "bound": "tensor" if tensor_path else "alu", "achieved": achieved,
+                         "peak": roof_peak, "unit": "TFLOP/s", "frac": achieved / roof_peak,
                          "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                         "peak_source": (f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"
+                                         if tensor_path else
+                                         "fp32 FMA peak: 148 SMs x 128 lanes x 2 flops x 1.965 GHz"),
                          "achieved_note": "8*d*E flops per unit x units per launch / CUDA-event time "
                                           "of the relkl_bwd_qkv call (dX zeroing included)"},
             "e2e": {"value": None if e2e_ms is None else total_fl / (e2e_ms * 1e-3) / 1e12,
