@@ -406,12 +406,19 @@ def main():
         rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
         rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
 
+    def stop_if_device_error(when):
+        # every rank takes this collective, so that all leave together on an error
+        code, where = rk.relkl_get_device_error(ws)
+        worst = int(max_over_ranks(float(code), dev))
+        if worst != 0:
+            if world > 1:
+                dist.destroy_process_group()
+            raise SystemExit(f"a device wait ran out {when} (this rank: code {code}, site {where})")
+
     for _ in range(args.warmup):
         step()
     barrier()
-    code, where = rk.relkl_get_device_error(ws)
-    if code != 0:
-        raise SystemExit(f"device wait ran out during warm-up (site {where})")
+    stop_if_device_error("during warm-up")
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -433,9 +440,7 @@ def main():
     ms = t_start.elapsed_time(t_end)
     fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
     bwd_ms = [b.elapsed_time(c) for _, b, c in ev]
-    code, where = rk.relkl_get_device_error(ws)
-    if code != 0:
-        raise SystemExit(f"device wait ran out in the timed region (site {where})")
+    stop_if_device_error("in the timed region")
     ms = max_over_ranks(ms, dev)
     peak_alloc = torch.cuda.max_memory_allocated(dev)
 
