@@ -68,3 +68,21 @@ def test_chain_workload_shapes_determinism_and_projection():
     # student hidden states differ from the teacher's by the configured noise
     diff = (a["h_s"].float() - a["h_t"].float()).std().item()
     assert 0.08 < diff < 0.12
+
+
+def test_bench_names_the_backward_kernel_the_library_launches():
+    # bench.py names the roofline kernel from N; the library picks it with kPairMinBlocks
+    import os
+    import re
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = open(os.path.join(root, "attention_relation_kl_b200", "csrc", "relkl_tc.cu")).read()
+    min_blocks = int(re.search(r"constexpr int kPairMinBlocks = (\d+);", src).group(1))
+    sys.path.insert(0, root)
+    import bench
+    for N in (128 * (min_blocks - 1), 128 * (min_blocks - 1) + 1, 32768):
+        w = workload.tiny_custom(N=N, d=128, dtype="bf16")
+        want = "relkl_bwd_pair_kernel" if (N + 127) // 128 >= min_blocks else "relkl_bwd_tc64_kernel"
+        assert bench.bwd_kernel_name(w) == want, N
+    assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=64, dtype="bf16")) == "relkl_bwd_tc_kernel"
+    assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=64, dtype="fp32")) == "relkl_bwd_simt_kernel"
