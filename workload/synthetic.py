@@ -90,6 +90,10 @@ CONFIGS: Dict[str, Workload] = {
     "gqa_llama3_n16k": Workload("gqa_llama3_n16k", B=2, H=32, H_kv=8, N=16384, d=128,
                                 dtype="bf16", causal=True, relations=("q", "k", "v"),
                                 rope_base=5e5, pi_factor=4.0, v_noise=0.05, seed=4),
+    # head dimension 64 (the smaller-head model class), otherwise the 32K shape
+    "d64_h32_n32k": Workload("d64_h32_n32k", B=1, H=32, H_kv=32, N=32768, d=64,
+                             dtype="bf16", causal=True, relations=("q", "k", "v"),
+                             rope_base=1e4, pi_factor=8.0, v_noise=0.1, seed=6),
 }
 
 SWEEP_N = (1024, 2048, 4096, 8192, 16384, 32768, 65536)
