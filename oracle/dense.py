@@ -43,6 +43,7 @@ from __future__ import annotations
 from typing import Dict, Iterable, Optional
 
 import numpy as np
+import torch
 
 __all__ = ["as_f64", "relation_logits", "allowed", "fwd_unit", "bwd_unit",
            "fwd_rows", "bwd_rows", "fwd", "bwd", "unit_loss"]
@@ -51,7 +52,10 @@ __all__ = ["as_f64", "relation_logits", "allowed", "fwd_unit", "bwd_unit",
 def as_f64(x) -> np.ndarray:
     """Exact float64 copy of a NumPy array or a (CPU) torch tensor."""
     if hasattr(x, "detach"):
-        x = x.detach().cpu().float().numpy()
+        x = x.detach().cpu()
+        if x.dtype in (torch.bfloat16, torch.float16):   # no NumPy type: widen exactly first
+            x = x.float()
+        x = x.numpy()
     return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
 
 
@@ -177,31 +181,48 @@ def bwd_rows(xt, xs, rows: Iterable[int], dkl=None, causal: bool = True,
     return s * (g_row @ xs + g_col.T @ xs)
 
 
+def _valid_len(lengths, b: int, N: int) -> int:
+    """Right padding: batch element b holds lengths[b] real tokens (clamped to
+    [0, N]); the rest are padding, excluded from every row distribution."""
+    return N if lengths is None else max(0, min(N, int(np.asarray(lengths)[b])))
+
+
 def fwd(xt, xs, causal: bool = True, scale: Optional[float] = None,
-        slab: int = 2048) -> Dict[str, np.ndarray]:
-    """Batched forward over [B, H, N, d]; each statistic comes back as [B, H, N]."""
+        slab: int = 2048, lengths=None) -> Dict[str, np.ndarray]:
+    """Batched forward over [B, H, N, d]; each statistic comes back as [B, H, N].
+
+    With ``lengths`` ([B]), batch element b is the sequence of its first
+    lengths[b] tokens; its padding rows come back as 0.
+    """
     xt, xs = as_f64(xt), as_f64(xs)
     B, H, N, _ = xt.shape
     out = {k: np.zeros((B, H, N)) for k in ("kl", "lse_t", "lse_s", "w", "m")}
     for b in range(B):
+        L = _valid_len(lengths, b, N)
+        if L == 0:
+            continue
         for h in range(H):
-            r = fwd_unit(xt[b, h], xs[b, h], causal, scale, slab)
+            r = fwd_unit(xt[b, h, :L], xs[b, h, :L], causal, scale, slab)
             for k in out:
-                out[k][b, h] = r[k]
+                out[k][b, h, :L] = r[k]
     return out
 
 
 def bwd(xt, xs, dkl=None, causal: bool = True, scale: Optional[float] = None,
-        slab: int = 2048) -> np.ndarray:
-    """Batched backward over [B, H, N, d]; ``dkl`` is [B, H, N] or None (1/N)."""
+        slab: int = 2048, lengths=None) -> np.ndarray:
+    """Batched backward over [B, H, N, d]; ``dkl`` is [B, H, N] or None (1/n per
+    row, n the sequence length: N, or lengths[b] with padding, whose rows get 0)."""
     xt, xs = as_f64(xt), as_f64(xs)
     B, H, N, _ = xt.shape
     g = None if dkl is None else as_f64(dkl).reshape(B, H, N)
     dx = np.zeros_like(xs)
     for b in range(B):
+        L = _valid_len(lengths, b, N)
+        if L == 0:
+            continue
         for h in range(H):
-            dx[b, h] = bwd_unit(xt[b, h], xs[b, h], None if g is None else g[b, h],
-                                causal, scale, slab)
+            dx[b, h, :L] = bwd_unit(xt[b, h, :L], xs[b, h, :L],
+                                    None if g is None else g[b, h, :L], causal, scale, slab)
     return dx
 
 

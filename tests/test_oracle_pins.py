@@ -295,3 +295,68 @@ def test_planted_mistakes_are_caught(monkeypatch):
         mod = type(dense)("oracle_mutant")
         exec(compile(src.replace(a, b), "oracle_mutant", "exec"), mod.__dict__)
         assert not _pins_pass(mod), f"planted mistake not caught: {name}"
+
+
+# ------------------------------------------------------- right padding
+
+def _padded_pair(B, H, N, d, seed):
+    gen = torch.Generator().manual_seed(seed)
+    xt = torch.randn(B, H, N, d, generator=gen, dtype=torch.float64)
+    xs = xt + 0.4 * torch.randn(B, H, N, d, generator=gen, dtype=torch.float64)
+    return xt, xs
+
+
+def test_lengths_equal_to_n_change_nothing():
+    xt, xs = _padded_pair(2, 2, 11, 4, 41)
+    full = np.array([11, 11])
+    for causal in (True, False):
+        a, b = dense.fwd(xt, xs, causal), dense.fwd(xt, xs, causal, lengths=full)
+        for k in a:
+            np.testing.assert_array_equal(a[k], b[k])
+        np.testing.assert_array_equal(dense.bwd(xt, xs, None, causal),
+                                      dense.bwd(xt, xs, None, causal, lengths=full))
+
+
+def test_padding_values_do_not_leak():
+    xt, xs = _padded_pair(3, 1, 12, 4, 42)
+    lengths = np.array([12, 7, 0])
+    yt, ys = xt.clone(), xs.clone()
+    for b, L in enumerate(lengths):
+        yt[b, :, L:] = 1e3
+        ys[b, :, L:] = -2e3
+    for causal in (True, False):
+        a, b = dense.fwd(xt, xs, causal, lengths=lengths), dense.fwd(yt, ys, causal, lengths=lengths)
+        np.testing.assert_array_equal(a["kl"], b["kl"])
+        assert np.all(a["kl"][1, :, 7:] == 0) and np.all(a["kl"][2] == 0)
+        da = dense.bwd(xt, xs, None, causal, lengths=lengths)
+        np.testing.assert_array_equal(da, dense.bwd(yt, ys, None, causal, lengths=lengths))
+        assert np.all(da[1, :, 7:] == 0) and np.all(da[2] == 0)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_lengths_match_torch_key_padding_mask(causal):
+    # independent formulation: full-length tensors, a key-padding mask on the
+    # columns, padded rows dropped from the loss, per-sequence mean over valid rows
+    B, H, N, d = 3, 2, 9, 4
+    xt, xs = _padded_pair(B, H, N, d, 43)
+    lengths = [9, 5, 1]
+    xs_var = xs.clone().requires_grad_(True)
+    s = 1.0 / np.sqrt(d)
+    loss = 0.0
+    kl_ref = torch.zeros(B, H, N, dtype=torch.float64)
+    for b in range(B):
+        L = lengths[b]
+        col_ok = torch.arange(N)[None, :] < L
+        ok = col_ok & (torch.tril(torch.ones(N, N, dtype=torch.bool)) if causal else True)
+        zt = (xt[b] @ xt[b].transpose(-1, -2) * s).masked_fill(~ok, float("-inf"))
+        zs = (xs_var[b] @ xs_var[b].transpose(-1, -2) * s).masked_fill(~ok, float("-inf"))
+        lt, ls = torch.log_softmax(zt[:, :L], -1), torch.log_softmax(zs[:, :L], -1)
+        kl = torch.nn.functional.kl_div(ls, lt, log_target=True, reduction="none").nan_to_num(0.0)
+        kl = kl.sum(-1)                        # [H, L]
+        kl_ref[b, :, :L] = kl.detach()
+        loss = loss + kl.sum() / L
+    loss.backward()
+    r = dense.fwd(xt, xs, causal, lengths=np.array(lengths))
+    np.testing.assert_allclose(r["kl"], kl_ref.numpy(), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(dense.bwd(xt, xs, None, causal, lengths=np.array(lengths)),
+                               xs_var.grad.numpy(), rtol=1e-9, atol=1e-12)
