@@ -99,6 +99,7 @@ relkl_status check_desc(const relkl_desc* d) {
   if (d->dtype != RELKL_BF16 && d->dtype != RELKL_FP32) return RELKL_ERR_INVALID;
   if (d->causal != 0 && d->causal != 1) return RELKL_ERR_INVALID;
   if (d->reserved != 0) return RELKL_ERR_INVALID;
+  if (d->lengths && !aligned(d->lengths, 4)) return RELKL_ERR_INVALID;
   if (!(d->scale >= 0.f) || !std::isfinite(d->scale)) return RELKL_ERR_INVALID;
   if (d->stride[3] != 1) return RELKL_ERR_INVALID;
   for (int i = 0; i < 3; ++i)
@@ -215,6 +216,7 @@ relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const*
     if ((st = encode_x(&s.tm_s, descs[r], xs[r])) != RELKL_OK) return st;
     s.B = descs[r].B;
     s.H = descs[r].H;
+    s.lengths = descs[r].lengths;
     s.unit_begin = ub;
     ub += static_cast<int>(n_units(descs[r]));
     ++seg;
@@ -247,6 +249,7 @@ relkl_status build_simt(int32_t n_rel, const relkl_desc* descs, const void* cons
     s.sn = descs[r].stride[2];
     s.B = descs[r].B;
     s.H = descs[r].H;
+    s.lengths = descs[r].lengths;
     s.unit_begin = ub;
     ub += static_cast<int>(n_units(descs[r]));
     ++seg;

@@ -22,6 +22,7 @@ struct TcSeg {
   float* stats;              // [B,H,N,4]
   const float* dkl;          // [B,H,N] or null (1/N)
   float* dx;                 // [B,H,N,d] float32
+  const int* lengths;        // [B] valid lengths (device) or null (all N)
   int B, H;
   int unit_begin;
   int pad_;
@@ -50,6 +51,7 @@ struct SimtSeg {
   float* stats;
   const float* dkl;
   float* dx;
+  const int* lengths;        // [B] valid lengths (device) or null (all N)
   int B, H;
   int unit_begin;
   int pad_;

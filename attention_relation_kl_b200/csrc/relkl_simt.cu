@@ -26,6 +26,7 @@ struct SimtUnit {
   const SimtSeg* seg;
   int64_t xoff;   // element offset of the unit's [N, d] slice in x
   int64_t row0;   // first row of the unit in [B,H,N] arrays
+  int L;          // valid rows and columns (its batch element's length, or N)
 };
 
 __device__ __forceinline__ SimtUnit simt_unit(const SimtParams& p, int u) {
@@ -39,6 +40,7 @@ __device__ __forceinline__ SimtUnit simt_unit(const SimtParams& p, int u) {
   out.seg = s;
   out.xoff = b * s->sb + h * s->sh;
   out.row0 = (static_cast<int64_t>(b) * s->H + h) * p.N;
+  out.L = s->lengths ? max(0, min(p.N, s->lengths[b])) : p.N;   // valid rows and columns
   return out;
 }
 
@@ -93,7 +95,7 @@ relkl_fwd_simt_kernel(const __grid_constant__ SimtParams p) {
       }
       zt[c] = at * sc;
       zs[c] = as * sc;
-      ok[c] = col < p.N && (!p.causal || col <= row);
+      ok[c] = row < U.L && col < U.L && (!p.causal || col <= row);
       if (ok[c]) mx = fmaxf(mx, fmaxf(zt[c], zs[c]));
     }
     // the 8 lanes of a row share one running maximum
@@ -121,7 +123,10 @@ relkl_fwd_simt_kernel(const __grid_constant__ SimtParams p) {
     C += __shfl_xor_sync(0xffffffffu, C, o);
     A += __shfl_xor_sync(0xffffffffu, A, o);
   }
-  if (cg == 0 && row < p.N) {
+  if (cg == 0 && row < p.N && row >= U.L) {   // padding row
+    S.kl[U.row0 + row] = 0.f;
+    reinterpret_cast<float4*>(S.stats)[U.row0 + row] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else if (cg == 0 && row < p.N) {
     const float lse_t = m_run + logf(St);
     const float l1 = log1pf(C / St);
     const float w = A / St;
@@ -152,11 +157,11 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
   stage_rows(xti, S.xt, p.is_bf16, U.xoff, S.sn, I * SB, p.N, d);
   stage_rows(xsi, S.xs, p.is_bf16, U.xoff, S.sn, I * SB, p.N, d);
   float lse_t = 0.f, lse_s = 0.f, mul = 0.f;
-  if (row < p.N) {
+  if (row < U.L) {
     const float4 st4 = reinterpret_cast<const float4*>(S.stats)[U.row0 + row];
     lse_t = st4.y;
     lse_s = st4.z;
-    mul = (S.dkl ? S.dkl[U.row0 + row] : 1.0f / static_cast<float>(p.N)) * sc;
+    mul = (S.dkl ? S.dkl[U.row0 + row] : 1.0f / static_cast<float>(U.L)) * sc;
   }
   // dX_I accumulator: this thread owns columns cg, cg+8, ... of row rr
   constexpr int MAXC = 128 / 8;
@@ -178,7 +183,7 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
         at = fmaf(xti[rr * pitch + k], xtj[jj * pitch + k], at);
         as = fmaf(xsi[rr * pitch + k], xsj[jj * pitch + k], as);
       }
-      const bool ok = row < p.N && col < p.N && (!p.causal || col <= row);
+      const bool ok = row < U.L && col < U.L && (!p.causal || col <= row);
       g[rr * (SB + 1) + jj] = ok ? mul * (expf(as * sc - lse_s) - expf(at * sc - lse_t)) : 0.f;
     }
     __syncthreads();

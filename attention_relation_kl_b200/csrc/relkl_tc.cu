@@ -89,6 +89,11 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
 
 // Row blocks of one work item: pass 0 is the longer block nblk-1-p, pass 1
 // (absent when both coincide) is block p.
+// Valid rows and columns of unit U: its batch element's length, or all N.
+__device__ __forceinline__ int unit_len(const TcParams& p, const Unit& U) {
+  const int* len = U.seg->lengths;
+  return len ? max(0, min(p.N, len[U.b])) : p.N;
+}
 __device__ __forceinline__ int item_passes(const TcParams& p, int pp) {
   return (pp == p.nblk - 1 - pp) ? 1 : 2;
 }
@@ -306,6 +311,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
         const int I = pass_block(p, pp, pass);
         const int row = I * BM + r;
         const int nT = n_col_tiles(p, I);
+        const int L = unit_len(p, U);
         float m_run = -INFINITY;
         // running sums, two float2 lanes each: S_t, C = sum(e_s - e_t), A = sum e_t (z_t - z_s)
         float2 S2[2], C2[2], A2[2];
@@ -327,7 +333,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
           if (lane == 0) mbar_arrive(TE(buf));
           ++nt;
           const int col0 = J * BN + wg * 32;
-          const bool need_mask = (p.causal && J == I) || (col0 + 32 > p.N);
+          const bool need_mask = (p.causal && J == I) || (col0 + 32 > L);
           if (!need_mask) {
             float m4[4];
 #pragma unroll
@@ -370,7 +376,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
             }
           } else {
             // diagonal or ragged tile: per-entry predicate
-            const int lim = p.causal ? min(row, p.N - 1) : p.N - 1;
+            const int lim = row >= L ? -1 : (p.causal ? min(row, L - 1) : L - 1);
             float mx = -INFINITY;
 #pragma unroll
             for (int k = 0; k < 32; ++k)
@@ -437,15 +443,18 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
           const float St = (Sx * a0 + o1.y * a1) + (o2.y * a2 + o3.y * a3);
           const float Ct = (Cx * a0 + o1.z * a1) + (o2.z * a2 + o3.z * a3);
           const float At = (Ax * a0 + o1.w * a1) + (o2.w * a2 + o3.w * a3);
-          if (row < p.N) {
+          const long long g = U.row0 + row;
+          if (row < L) {
             const float mz = M * p.scale;
             const float lse_t = mz + logf(St);
             const float rc = Ct / St;
             const float l1 = log1pf(rc);
             const float w = p.scale * At / St;
-            const long long g = U.row0 + row;
             U.seg->kl[g] = w + l1;
             reinterpret_cast<float4*>(U.seg->stats)[g] = make_float4(mz, lse_t, lse_t + l1, w);
+          } else if (row < p.N) {   // padding row
+            U.seg->kl[g] = 0.f;
+            reinterpret_cast<float4*>(U.seg->stats)[g] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
         ++nm;
@@ -762,16 +771,17 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
         const int I = pass_block(p, pp, pass);
         const int row = I * BM + r;
-        const bool rvalid = row < p.N;
+        const int L = unit_len(p, U);
+        const bool rvalid = row < L;
         float bt = 0.f, bs = 0.f, mul = 0.f;
         if (rvalid) {
           const float4 st4 = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + row];
           bt = -st4.y * kLog2e;
           bs = -st4.z * kLog2e;
-          const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(p.N);
+          const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(L);
           mul = up * p.scale;   // the logit scale of dX_s is folded into G
         }
-        const int lim = !rvalid ? -1 : (p.causal ? min(row, p.N - 1) : p.N - 1);
+        const int lim = !rvalid ? -1 : (p.causal ? min(row, L - 1) : L - 1);
         const int nT = n_col_tiles(p, I);
         for (int J = 0; J < nT; ++J) {
           ok = mbar_wait(S_FULL, ns & 1, wc, W_SM_S_FULL);
@@ -1175,16 +1185,17 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
       for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
         const int I = pass_block(p, pp, pass);
         const int row = I * BM + r;
-        const bool rvalid = row < p.N;
+        const int L = unit_len(p, U);
+        const bool rvalid = row < L;
         float bt = 0.f, bs = 0.f, mul = 0.f;
         if (rvalid) {
           const float4 st4 = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + row];
           bt = -st4.y * kLog2e;
           bs = -st4.z * kLog2e;
-          const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(p.N);
+          const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(L);
           mul = up * p.scale;   // the logit scale of dX_s is folded into G
         }
-        const int lim = !rvalid ? -1 : (p.causal ? min(row, p.N - 1) : p.N - 1);
+        const int lim = !rvalid ? -1 : (p.causal ? min(row, L - 1) : L - 1);
         const int nT = n_col_tiles64(p, I);
         const float2 sl2v = make_float2(sl2, sl2), btv = make_float2(bt, bt),
                      bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
@@ -1657,22 +1668,23 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         const bool has1 = R0 + 1 < p.nblk;
         const int nT0 = n_col_tiles64(p, R0);
         const int nT = has1 ? n_col_tiles64(p, R0 + 1) : nT0;
+        const int L = unit_len(p, U);
         // per-row constants of both row blocks
         float bt[2], bs[2], mul[2];
         int lim[2];
 #pragma unroll
         for (int rs = 0; rs < 2; ++rs) {
           const int row = (R0 + rs) * BM + r;
-          const bool rvalid = row < p.N && (rs == 0 || has1);
+          const bool rvalid = row < L && (rs == 0 || has1);
           bt[rs] = bs[rs] = mul[rs] = 0.f;
           if (rvalid) {
             const float4 st4 = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + row];
             bt[rs] = -st4.y * kLog2e;
             bs[rs] = -st4.z * kLog2e;
-            const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(p.N);
+            const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(L);
             mul[rs] = up * p.scale;   // the logit scale of dX_s is folded into G
           }
-          lim[rs] = !rvalid ? -1 : (p.causal ? min(row, p.N - 1) : p.N - 1);
+          lim[rs] = !rvalid ? -1 : (p.causal ? min(row, L - 1) : L - 1);
         }
         const float2 sl2v = make_float2(sl2, sl2), m1 = make_float2(-1.f, -1.f);
         for (int J = 0; ok && J < nT; ++J) {

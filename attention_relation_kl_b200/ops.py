@@ -27,7 +27,18 @@ __all__ = ["relkl_fwd", "relkl_bwd", "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_wo
 _DTYPES = {torch.bfloat16: _abi.RELKL_BF16, torch.float32: _abi.RELKL_FP32}
 
 
-def make_desc(x: torch.Tensor, causal: bool = True, scale: float = 0.0) -> relkl_desc:
+def _lengths_ptr(lengths: Optional[torch.Tensor], x: torch.Tensor) -> Optional[int]:
+    """Device pointer of per-batch valid lengths (int32 [B] on x's device), or None."""
+    if lengths is None:
+        return None
+    if (lengths.dtype != torch.int32 or lengths.dim() != 1 or lengths.shape[0] != x.shape[0]
+            or not lengths.is_contiguous() or lengths.device != x.device):
+        raise ValueError("lengths must be a contiguous int32 [B] tensor on the inputs' device")
+    return int(lengths.data_ptr())
+
+
+def make_desc(x: torch.Tensor, causal: bool = True, scale: float = 0.0,
+              lengths: Optional[torch.Tensor] = None) -> relkl_desc:
     if x.dim() != 4:
         raise ValueError("expected a [B, H, N, d] tensor")
     if x.dtype not in _DTYPES:
@@ -41,6 +52,7 @@ def make_desc(x: torch.Tensor, causal: bool = True, scale: float = 0.0) -> relkl
     d.causal = 1 if causal else 0
     d.scale = float(scale)
     d.reserved = 0
+    d.lengths = _lengths_ptr(lengths, x)
     return d
 
 
@@ -94,8 +106,10 @@ def _arr(vals, ctype=ctypes.c_void_p):
 
 def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bool = True,
                   scale: float = 0.0, *, out: Optional[Sequence[Tuple[torch.Tensor, torch.Tensor]]] = None,
-                  ws: Optional[torch.Tensor] = None, stream=None):
-    """Forward over 1..3 relations in one launch.  Returns [(kl, stats)] per relation."""
+                  ws: Optional[torch.Tensor] = None, stream=None,
+                  lengths: Optional[torch.Tensor] = None):
+    """Forward over 1..3 relations in one launch.  Returns [(kl, stats)] per relation.
+    ``lengths``: optional int32 [B] valid lengths (right padding), shared by the relations."""
     n = len(pairs)
     if not 1 <= n <= 3:
         raise ValueError("1 to 3 relations per call")
@@ -107,7 +121,7 @@ def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bo
         _cuda(xs, "x_s")
         if xt.shape != xs.shape or xt.stride() != xs.stride() or xt.dtype != xs.dtype:
             raise ValueError("teacher and student must share shape, strides and dtype")
-        descs[r] = make_desc(xt, causal, scale)
+        descs[r] = make_desc(xt, causal, scale, lengths)
         B, H, N, _ = xt.shape
         if out is not None:
             kl, st = out[r]
@@ -127,7 +141,8 @@ def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bo
 def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Sequence[torch.Tensor],
                   dkl: Optional[Sequence[Optional[torch.Tensor]]] = None, causal: bool = True,
                   scale: float = 0.0, *, out: Optional[Sequence[torch.Tensor]] = None,
-                  ws: Optional[torch.Tensor] = None, stream=None) -> List[torch.Tensor]:
+                  ws: Optional[torch.Tensor] = None, stream=None,
+                  lengths: Optional[torch.Tensor] = None) -> List[torch.Tensor]:
     """Backward over 1..3 relations in one launch.  Returns dX_s per relation (float32)."""
     n = len(pairs)
     if not 1 <= n <= 3 or len(stats) != n:
@@ -140,7 +155,7 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
         _cuda(xs, "x_s")
         if xt.shape != xs.shape or xt.stride() != xs.stride() or xt.dtype != xs.dtype:
             raise ValueError("teacher and student must share shape, strides and dtype")
-        descs[r] = make_desc(xt, causal, scale)
+        descs[r] = make_desc(xt, causal, scale, lengths)
         if not stats[r].is_contiguous() or stats[r].dtype != torch.float32:
             raise ValueError("stats must be contiguous float32 [B, H, N, 4]")
         if dkl is not None and dkl[r] is not None and (not dkl[r].is_contiguous()
@@ -162,24 +177,28 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
 
 def relkl_fwd(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True, scale: float = 0.0, *,
               kl: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
-              ws: Optional[torch.Tensor] = None, stream=None):
+              ws: Optional[torch.Tensor] = None, stream=None,
+              lengths: Optional[torch.Tensor] = None):
     """Per-row KL [B,H,N] and statistics [B,H,N,4] of one relation."""
     out = None if kl is None else [(kl, stats)]
-    return relkl_fwd_qkv([(x_t, x_s)], causal, scale, out=out, ws=ws, stream=stream)[0]
+    return relkl_fwd_qkv([(x_t, x_s)], causal, scale, out=out, ws=ws, stream=stream,
+                         lengths=lengths)[0]
 
 
 def relkl_bwd(x_t: torch.Tensor, x_s: torch.Tensor, stats: torch.Tensor,
               dkl: Optional[torch.Tensor] = None, causal: bool = True, scale: float = 0.0, *,
               dx_s: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-              stream=None) -> torch.Tensor:
-    """dL/dX_s (float32) with L = sum_i dkl_i kl_i (dkl=None: 1/N per row)."""
+              stream=None, lengths: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """dL/dX_s (float32) with L = sum_i dkl_i kl_i (dkl=None: 1/N per row, 1/L_b with lengths)."""
     return relkl_bwd_qkv([(x_t, x_s)], [stats], None if dkl is None else [dkl], causal, scale,
-                         out=None if dx_s is None else [dx_s], ws=ws, stream=stream)[0]
+                         out=None if dx_s is None else [dx_s], ws=ws, stream=stream,
+                         lengths=lengths)[0]
 
 
 def relkl_fwd_noalloc(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,
                       scale: float = 0.0, *, kl: Optional[torch.Tensor] = None,
-                      stats: Optional[torch.Tensor] = None, stream=None):
+                      stats: Optional[torch.Tensor] = None, stream=None,
+                      lengths: Optional[torch.Tensor] = None):
     """relkl_fwd for callers that cannot provide a device workspace.
 
     The library call itself allocates nothing: its scratch lives in a static
@@ -191,7 +210,7 @@ def relkl_fwd_noalloc(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,
     _cuda(x_s, "x_s")
     if x_t.shape != x_s.shape or x_t.stride() != x_s.stride() or x_t.dtype != x_s.dtype:
         raise ValueError("teacher and student must share shape, strides and dtype")
-    desc = make_desc(x_t, causal, scale)
+    desc = make_desc(x_t, causal, scale, lengths)
     B, H, N, _ = x_t.shape
     if kl is None:
         kl = torch.empty((B, H, N), dtype=torch.float32, device=x_t.device)
@@ -220,24 +239,25 @@ class RelationKL(torch.autograd.Function):
     """kl rows of one relation; backward runs relkl_bwd (teacher is frozen)."""
 
     @staticmethod
-    def forward(ctx, x_t, x_s, causal=True, scale=0.0):
-        kl, stats = relkl_fwd(x_t.detach(), x_s.detach(), causal, scale)
+    def forward(ctx, x_t, x_s, causal=True, scale=0.0, lengths=None):
+        kl, stats = relkl_fwd(x_t.detach(), x_s.detach(), causal, scale, lengths=lengths)
         ctx.save_for_backward(x_t, x_s, stats)
-        ctx.causal, ctx.scale = causal, scale
+        ctx.causal, ctx.scale, ctx.lengths = causal, scale, lengths
         return kl
 
     @staticmethod
     def backward(ctx, dkl):
         x_t, x_s, stats = ctx.saved_tensors
         dx = relkl_bwd(x_t.detach(), x_s.detach(), stats, dkl.contiguous().float(), ctx.causal,
-                       ctx.scale)
-        return None, dx, None, None
+                       ctx.scale, lengths=ctx.lengths)
+        return None, dx, None, None, None
 
 
 def relation_kl(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,
-                scale: float = 0.0) -> torch.Tensor:
-    """Differentiable per-row KL(R_t || R_s) of one relation, shape [B, H, N]."""
-    return RelationKL.apply(x_t, x_s, causal, scale)
+                scale: float = 0.0, lengths: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Differentiable per-row KL(R_t || R_s) of one relation, shape [B, H, N]
+    (rows past ``lengths[b]`` are padding: kl 0, no gradient)."""
+    return RelationKL.apply(x_t, x_s, causal, scale, lengths)
 
 
 # ------------------------------------------------ chain rule to the weights

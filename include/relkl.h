@@ -74,6 +74,13 @@ typedef struct {
   int32_t causal;    /* 1: row i sees columns j <= i; 0: every column       */
   float scale;       /* logit scale; 0 means 1/sqrt(d)                      */
   int32_t reserved;  /* must be 0                                           */
+  /* Optional right padding: DEVICE pointer to B int32 valid lengths (NULL: all
+   * N rows valid).  For batch b, rows and columns >= L_b = clamp(lengths[b],
+   * 0, N) are padding: no row distribution includes them, their kl rows and
+   * stats are 0, their dX_s rows are 0, and the default upstream gradient of
+   * a valid row is 1/L_b.  Read on the device; must stay valid until the
+   * queued work has finished; 4-byte aligned.                               */
+  const int32_t* lengths;
 } relkl_desc;
 
 /* Bytes of device workspace a call needs (for every entry point, any desc):

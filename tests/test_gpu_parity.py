@@ -247,3 +247,64 @@ def test_config_sweep_n64k():
     w = workload.sweep_config(65536)
     units = [("q", 0, 0), ("k", 0, 9), ("v", 0, 31)]
     _sampled(w, units, dx_units={("k", 0, 9)})
+
+
+# ------------------------------------------------------ right padding
+
+def _padded_inputs(B, H, N, d, dtype, seed, lengths):
+    w = workload.tiny_custom(N=N, d=d, dtype=dtype, seed=seed, pi_factor=4.0, B=B, H=H)
+    xt, xs = workload.generate(w)["q"]
+    xt, xs = xt.clone(), xs.clone()
+    for b, L in enumerate(lengths):          # garbage in the padding must not leak
+        xt[b, :, L:] = 30.0
+        xs[b, :, L:] = -45.0
+    return xt, xs
+
+
+@pytest.mark.parametrize("B,H,N,d,dtype,causal,lengths,path", [
+    (3, 2, 300, 128, "bf16", True, [300, 263, 0], 1),
+    (3, 2, 300, 128, "bf16", False, [300, 177, 1], 1),
+    (2, 1, 513, 64, "bf16", False, [513, 200], 1),
+    (2, 1, 4200, 128, "bf16", True, [4200, 3001], 1),      # pair backward
+    (2, 1, 4200, 128, "bf16", False, [2100, 4200], 1),
+    (2, 2, 150, 64, "fp32", True, [150, 61], 2),           # CUDA-core path
+    (2, 2, 150, 64, "fp32", False, [97, 150], 2),
+])
+def test_padded_lengths(B, H, N, d, dtype, causal, lengths, path):
+    xt, xs = _padded_inputs(B, H, N, d, dtype, N + d + len(lengths), lengths)
+    lens = torch.tensor(lengths, dtype=torch.int32)
+    gt, gs, gl = xt.cuda(), xs.cuda(), lens.cuda()
+    assert rk.relkl_path_for(gt, causal) == path
+    kl, st = rk.relkl_fwd(gt, gs, causal, lengths=gl)
+    dx = rk.relkl_bwd(gt, gs, st, None, causal, lengths=gl)
+    torch.cuda.synchronize()
+    _device_ok()
+    ref = dense.fwd(xt, xs, causal, lengths=lengths)
+    assert_kl(to_np(kl), ref["kl"])
+    for b, L in enumerate(lengths):
+        assert np.all(to_np(kl[b, :, L:]) == 0) and np.all(to_np(st[b, :, L:]) == 0)
+        if L:
+            assert_stats(to_np(st[b, :, :L]), {k: v[b, :, :L] for k, v in ref.items()})
+    tol = DX_TOL_BF16 if path == 1 else DX_TOL_FP32
+    ref_dx = dense.bwd(xt, xs, None, causal, lengths=lengths)
+    assert_dx(to_np(dx), ref_dx, tol)
+    for b, L in enumerate(lengths):
+        assert np.all(to_np(dx[b, :, L:]) == 0)
+
+
+def test_fused_qkv_gqa_padded():
+    g = workload.Workload("gqa_pad", B=2, H=4, H_kv=2, N=320, d=128, dtype="bf16", causal=True,
+                          relations=("q", "k", "v"), rope_base=5e5, pi_factor=4.0, v_noise=0.05,
+                          seed=29)
+    x = workload.generate(g)
+    lengths = [320, 190]
+    lens = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+    pairs = [(x[r][0].cuda(), x[r][1].cuda()) for r in "qkv"]
+    outs = rk.relkl_fwd_qkv(pairs, lengths=lens)
+    dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], lengths=lens)
+    torch.cuda.synchronize()
+    _device_ok()
+    for r, (kl, _), dx in zip("qkv", outs, dxs):
+        ref = dense.fwd(*x[r], lengths=lengths)
+        assert_kl(to_np(kl), ref["kl"], what=f"kl[{r}]")
+        assert_dx(to_np(dx), dense.bwd(*x[r], lengths=lengths), DX_TOL_BF16)
