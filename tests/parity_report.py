@@ -60,6 +60,49 @@ def run_small(out):
         out.append((name, path, "all rows", *m))
 
 
+def run_padded(out):
+    """Right-padded batches (garbage in the padding) on every kernel family."""
+    for (B, H, N, d, dtype, causal, lengths) in [(3, 2, 300, 128, "bf16", True, [300, 263, 0]),
+                                                 (3, 2, 300, 128, "bf16", False, [300, 177, 1]),
+                                                 (2, 1, 4200, 128, "bf16", True, [4200, 3001]),
+                                                 (2, 2, 150, 64, "fp32", False, [97, 150])]:
+        w = workload.tiny_custom(N=N, d=d, dtype=dtype, seed=N + d, causal=causal, B=B, H=H)
+        xt, xs = workload.generate(w)["q"]
+        xt, xs = xt.clone(), xs.clone()
+        for b, L in enumerate(lengths):
+            xt[b, :, L:] = 30.0
+            xs[b, :, L:] = -45.0
+        gl = torch.tensor(lengths, dtype=torch.int32, device="cuda")
+        gt, gs = xt.cuda(), xs.cuda()
+        path = "tcgen05" if rk.relkl_path_for(gt, causal) == 1 else "CUDA-core fp32"
+        kl, st = rk.relkl_fwd(gt, gs, causal, lengths=gl)
+        dx = rk.relkl_bwd(gt, gs, st, None, causal, lengths=gl)
+        torch.cuda.synchronize()
+        tol = DX_TOL_BF16 if path == "tcgen05" else DX_TOL_FP32
+        m = margins(to_np(kl), dense.fwd(xt, xs, causal, lengths=lengths)["kl"], to_np(dx),
+                    dense.bwd(xt, xs, None, causal, lengths=lengths), tol)
+        out.append((f"padded N={N} d={d} {'causal' if causal else 'full'} {dtype} lengths={lengths}",
+                    path, "all rows", *m))
+
+
+def run_chain(out):
+    """dW_q, dW_k, dW_v of the small chain workload (kl columns: not applicable)."""
+    from oracle import chain
+    cw = workload.CHAIN_CONFIGS["chain_small"]
+    c = workload.generate_chain(cw)
+    pairs = {r: (c["x"][r][0].cuda(), c["x"][r][1].cuda()) for r in "qkv"}
+    got = rk.student_weight_grads(pairs, c["h_s"].cuda(), cw.rope_base, 1.0 / cw.pi_factor,
+                                  cw.causal)
+    torch.cuda.synchronize()
+    ref = chain.projection_grads(c["x"], c["h_s"], c["pos_s"].numpy(), cw.rope_base,
+                                 causal=cw.causal)
+    for r in "qkv":
+        g, w = to_np(got[r]), ref[r]
+        rel = float(np.abs(g - w).max() / np.abs(w).max())
+        out.append((f"chain_small dW_{r} [{w.shape[0]}x{w.shape[1]}]", "RoPE bwd + cuBLAS GEMM",
+                    "every weight", float("nan"), float("nan"), rel, rel / DX_TOL_BF16))
+
+
 def run_full(out):
     for cfg, units in (("llama2_h32_n4k", [("q", 0, 0), ("v", 0, 31)]),
                        ("gqa_llama3_n16k", [("k", 0, 3), ("v", 1, 7)]),
@@ -86,6 +129,8 @@ def main():
     out = []
     t0 = time.time()
     run_small(out)
+    run_padded(out)
+    run_chain(out)
     if "--full" in sys.argv:
         run_full(out)
     print(f"# Parity margins against the float64 oracle ({torch.cuda.get_device_name(0)})\n")
