@@ -50,7 +50,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + ".tmp"
     cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
-           *[os.path.join(CSRC, f) for f in SOURCES], "-lcublas", "-o", tmp]
+           *[os.path.join(CSRC, f) for f in SOURCES], "-lcublas", "-ldl", "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)

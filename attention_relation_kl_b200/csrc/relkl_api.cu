@@ -10,6 +10,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/relkl.h"
 #include "relkl_device.cuh"
@@ -40,6 +41,17 @@ relkl_status cuda_fail(cudaError_t e) {
   g_last_cuda = static_cast<int32_t>(e);
   return RELKL_ERR_CUDA;
 }
+
+// NVTX range over the host side of one entry point (validation, descriptor
+// encoding, launches), so that a profiler timeline shows which call queued
+// which kernels.  NVTX3 is header-only: without an attached tool the push and
+// pop are a load and a branch.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // cuTensorMapEncodeTiled, fetched from the driver through the runtime so the
 // library needs no link-time dependency on libcuda.
@@ -302,6 +314,7 @@ int32_t relkl_path_for(const relkl_desc* desc) {
 relkl_status relkl_fwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
                            const void* const* x_s, float* const* kl, float* const* stats,
                            void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("relkl_fwd_qkv");
   bool empty = false;
   relkl_status s = check_multi(n_rel, descs, x_t, x_s, &empty);
   if (s != RELKL_OK || empty) return s;
@@ -334,6 +347,7 @@ relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* c
                            const void* const* x_s, const float* const* stats,
                            const float* const* dkl, float* const* dx_s, void* ws,
                            size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("relkl_bwd_qkv");
   bool empty = false;
   relkl_status s = check_multi(n_rel, descs, x_t, x_s, &empty);
   if (s != RELKL_OK || empty) return s;
@@ -436,6 +450,7 @@ int32_t relkl_last_cuda_error(void) { return g_last_cuda; }
 relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const float* dx_post,
                             const relkl_rope* rope, int32_t out_dtype, void* dx_pre,
                             void* stream) {
+  NvtxRange nvtx_range("relkl_rope_bwd");
   if (!rope || B < 0 || H < 0 || N < 0 || d < 2 || d > 512 || (d & 1)) return RELKL_ERR_INVALID;
   if (out_dtype != RELKL_BF16 && out_dtype != RELKL_FP32) return RELKL_ERR_INVALID;
   if (rope->reserved != 0 || (rope->apply != 0 && rope->apply != 1)) return RELKL_ERR_INVALID;
@@ -455,6 +470,7 @@ relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const fl
 
 relkl_status relkl_weight_grad(int64_t rows, int32_t D, int32_t cols, const void* h,
                                const void* dx_pre, float* dw, void* stream) {
+  NvtxRange nvtx_range("relkl_weight_grad");
   if (rows < 1 || rows > 0x7fffffffLL || D < 1 || cols < 1 || (D % 8) || (cols % 8))
     return RELKL_ERR_INVALID;
   if (!h || !dx_pre || !dw || !aligned(h, 16) || !aligned(dx_pre, 16) || !aligned(dw, 16))
@@ -478,8 +494,34 @@ relkl_status relkl_weight_grad(int64_t rows, int32_t D, int32_t cols, const void
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RELKL_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-void* g_noalloc_addr[64];
+// One slot per device index: the array's device address and the context it
+// was looked up in.  A context torn down and created again (cudaDeviceReset,
+// or a reset after a sticky error) loads the module again, possibly at another
+// address, so a slot is only reused while the device's current context is the
+// one recorded in it.
+struct NoallocSlot {
+  CUcontext ctx;
+  void* addr;
+};
+NoallocSlot g_noalloc[64];
 std::mutex g_noalloc_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn g_ctx_current = nullptr;
+std::once_flag g_ctx_once;
+
+CUcontext current_context() {
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+  });
+  CUcontext c = nullptr;
+  if (g_ctx_current && g_ctx_current(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
 
 relkl_status noalloc_scratch(void** out) {
   int dev = 0;
@@ -487,13 +529,16 @@ relkl_status noalloc_scratch(void** out) {
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= 64) return RELKL_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
+  NoallocSlot& slot = g_noalloc[dev];
+  const CUcontext ctx = current_context();
+  if (!slot.addr || ctx != slot.ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) return cuda_fail(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
-    g_noalloc_addr[dev] = p;
+    slot.addr = p;
+    slot.ctx = current_context();   // the lookup made the device's context current
   }
-  *out = g_noalloc_addr[dev];
+  *out = slot.addr;
   return RELKL_OK;
 }
 }  // namespace
@@ -501,6 +546,7 @@ relkl_status noalloc_scratch(void** out) {
 extern "C" relkl_status relkl_fwd_noalloc(const relkl_desc* desc, const void* x_t,
                                           const void* x_s, float* kl, float* stats,
                                           void* stream) {
+  NvtxRange nvtx_range("relkl_fwd_noalloc");
   const void* xt[1] = {x_t};
   const void* xs[1] = {x_s};
   bool empty = false;

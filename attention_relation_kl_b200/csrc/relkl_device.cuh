@@ -324,42 +324,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x for a pair of arguments on the FMA pipe instead of MUFU, for x <= 0
-// (arguments below -125 are clamped; their results are < 2^-125).
-// Cody and Waite's reduction x = n + f with n = rint(x), f in [-1/2, 1/2]
-// (n comes from adding 1.5 * 2^23, which leaves rint(x) in the low mantissa
-// bits), a polynomial p(f) ~ 2^f with minimax relative error fitted by
-// csrc/fit_exp2_poly.py, and n added to p's exponent field with one integer
-// multiply-add.  DEG 5: relative error 1.8e-7 (float32 evaluation, on par with
-// ex2.approx); DEG 3: 1.0e-4.
-template <int DEG>
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  static_assert(DEG == 3 || DEG == 5, "fitted degrees are 3 and 5");
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
-  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
-  float2 p;
-  if constexpr (DEG == 5) {
-    p = __ffma2_rn(make_float2(1.326627913e-03f, 1.326627913e-03f), f,
-                   make_float2(9.671512060e-03f, 9.671512060e-03f));
-    p = __ffma2_rn(p, f, make_float2(5.550728366e-02f, 5.550728366e-02f));
-    p = __ffma2_rn(p, f, make_float2(2.402224243e-01f, 2.402224243e-01f));
-    p = __ffma2_rn(p, f, make_float2(6.931470037e-01f, 6.931470037e-01f));
-  } else {
-    p = __ffma2_rn(make_float2(5.502312258e-02f, 5.502312258e-02f), f,
-                   make_float2(2.422109395e-01f, 2.422109395e-01f));
-    p = __ffma2_rn(p, f, make_float2(6.932800412e-01f, 6.932800412e-01f));
-  }
-  p = __ffma2_rn(p, f, make_float2(1.0f, 1.0f));
-  // the low 9 bits of t's pattern hold n (two's complement); shifted by 23
-  // they land on the exponent field (unsigned arithmetic wraps mod 2^32)
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 __device__ __forceinline__ float2 ex2_approx2(float2 x) {
   return make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }

@@ -7,21 +7,24 @@
 // in the backward pass (Phase 2), where G = dkl (R_s - R_t) and
 // dX_s = s (G + G^T) X_s.
 //
-// Both kernels are persistent (one CTA per SM, static schedule) and
+// Every kernel here is persistent (one CTA per SM, static schedule) and
 // warp-specialised:
-//   * one TMA warp streams 128-row bf16 tiles of X_t and X_s into 128-byte
-//     swizzled shared memory (the row block I stays resident, column blocks J
-//     pass through a two-stage ring);
-//   * one MMA warp issues tcgen05.mma (kind::f16, M=128) whose fp32
+//   * one TMA warp streams bf16 tiles of X_t and X_s into 128-byte swizzled
+//     shared memory (the row blocks of a work item stay resident, column tiles
+//     pass through rings);
+//   * one or two MMA warps issue tcgen05.mma (kind::f16, M=128) whose fp32
 //     accumulators live in tensor memory: the teacher and student logit tiles
-//     side by side, and in the backward also dX_I += G X_s[J] and
-//     P = G^T X_s[I];
-//   * two "row" warpgroups read the logit tiles from TMEM (one column half
-//     each) and do the per-entry work: the shared-max online softmax and KL
-//     sums in the forward, the gradient tile G (bf16, written to shared
-//     memory as an MMA operand) in the backward;
-//   * in the backward an epilogue warpgroup adds P into dX[J] and, at the end
-//     of a row block, the dX_I accumulator into dX[I] with float32 atomics.
+//     side by side, and in the backward also the row-side product
+//     dX_I += G X_s[J] and the column-side product P = G^T X_s[I] (or its
+//     transpose);
+//   * four "row" warpgroups read the logit tiles from TMEM (each owns a slice
+//     of the tile's columns) and do the per-entry work: the shared-max online
+//     softmax and KL sums in the forward, the gradient tile G (bf16, written
+//     to shared memory as an MMA operand) in the backward;
+//   * in the backward an epilogue warpgroup stages the column-side product and,
+//     at the end of a row block, the dX_I accumulator as 32 x 32 fp32 boxes in
+//     shared memory and adds them into dX with TMA bulk-tensor reduce-adds
+//     (the additions happen in L2).
 //
 // Work items pair row block p with row block nblk-1-p of the same unit, so
 // every causal item holds nblk+1 column tiles and the static round-robin over
@@ -45,24 +48,6 @@ constexpr int BM = 128;        // rows of a row block (TMEM lanes)
 constexpr int BN = 128;        // columns of a logit tile
 constexpr int BOX = 128 * 128;  // bytes of one 128-row x 64-col bf16 box
 constexpr float kLog2e = 1.4426950408889634f;
-
-// Which column pairs take 2^x on the FMA pipe (exp2_poly2) instead of MUFU.
-// Measured on B200: MUFU ex2 costs 8 clk per warp instruction (4 lanes/clk per
-// SMSP); the degree-3 packed polynomial costs ~19.5 clk per pair of exps on
-// the FMA pipe (FFMA2 is 2 clk, not 1), and the FMA pipe already carries the
-// exp arguments, differences and accumulations of every entry.  In both
-// kernels moving exps off MUFU therefore lengthened the exp pass, so no pair
-// is offloaded unless RELKL_EXP2_POLY is defined (forward: 4 of 16 pairs with
-// the degree-5 fit; backward: 3 of 8 pairs with the degree-3 fit).
-#ifdef RELKL_EXP2_POLY
-__host__ __device__ constexpr bool fwd_poly_pair(int pair) { return (pair & 3) == 3; }
-__host__ __device__ constexpr bool bwd_poly_pair(int pair) {
-  return (pair & 7) == 2 || (pair & 7) == 5 || (pair & 7) == 7;
-}
-#else
-__host__ __device__ constexpr bool fwd_poly_pair(int) { return false; }
-__host__ __device__ constexpr bool bwd_poly_pair(int) { return false; }
-#endif
 
 constexpr unsigned long long kDrainNs = 200000000ull;  // 0.2 s for in-flight copies
 
@@ -361,14 +346,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
               const float2 sv = make_float2(s[k], s[k + 1]);
               const float2 at = __ffma2_rn(tv, sl2v, nbv);
               const float2 as = __ffma2_rn(sv, sl2v, nbv);
-              float2 et, es;
-              if (fwd_poly_pair(k >> 1)) {
-                et = exp2_poly2<5>(at);
-                es = exp2_poly2<5>(as);
-              } else {
-                et = ex2_approx2(at);
-                es = ex2_approx2(as);
-              }
+              const float2 et = ex2_approx2(at), es = ex2_approx2(as);
               const int a = (k >> 1) & 1;
               S2[a] = __fadd2_rn(S2[a], et);
               C2[a] = __fadd2_rn(C2[a], __ffma2_rn(et, m1, es));
@@ -807,14 +785,7 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
           for (int k = 0; k < 32; k += 2) {
             const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
             const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
-            float2 et, es;
-            if (bwd_poly_pair(k >> 1)) {
-              et = exp2_poly2<3>(at);
-              es = exp2_poly2<3>(as);
-            } else {
-              et = ex2_approx2(at);
-              es = ex2_approx2(as);
-            }
+            const float2 et = ex2_approx2(at), es = ex2_approx2(as);
             float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
             if (need_mask) {
               g.x = (col0 + k <= lim) ? g.x : 0.f;
@@ -1222,14 +1193,7 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
           for (int k = 0; k < 16; k += 2) {
             const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
             const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
-            float2 et, es;
-            if (bwd_poly_pair(k >> 1)) {
-              et = exp2_poly2<3>(at);
-              es = exp2_poly2<3>(as);
-            } else {
-              et = ex2_approx2(at);
-              es = ex2_approx2(as);
-            }
+            const float2 et = ex2_approx2(at), es = ex2_approx2(as);
             float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
             if (need_mask) {
               g.x = (col0 + k <= lim) ? g.x : 0.f;

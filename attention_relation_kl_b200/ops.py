@@ -71,6 +71,18 @@ def _cuda(t: torch.Tensor, name: str) -> None:
         raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
 
 
+def _check_out(t: torch.Tensor, shape, name: str, device: torch.device) -> None:
+    """A caller-provided output must be exactly what the kernels write through
+    the raw pointer: contiguous float32 of the given shape on the inputs' device."""
+    if t is None:
+        raise ValueError(f"{name} must be given")
+    if (t.dtype != torch.float32 or tuple(t.shape) != tuple(shape) or not t.is_contiguous()
+            or t.device != device):
+        raise ValueError(f"{name} must be a contiguous float32 tensor of shape {tuple(shape)} "
+                         f"on {device} (got {t.dtype} {tuple(t.shape)} on {t.device}, "
+                         f"contiguous={t.is_contiguous()})")
+
+
 _WS: Dict[int, torch.Tensor] = {}
 
 
@@ -79,8 +91,10 @@ def relkl_workspace_bytes() -> int:
 
 
 def relkl_workspace_init(ws: torch.Tensor, stream=None) -> None:
-    check(_abi.lib().relkl_workspace_init(_ptr(ws), ws.numel() * ws.element_size(),
-                                          _stream(ws.device, stream)), "relkl_workspace_init")
+    with torch.cuda.device(ws.device):
+        code = _abi.lib().relkl_workspace_init(_ptr(ws), ws.numel() * ws.element_size(),
+                                               _stream(ws.device, stream))
+    check(code, "relkl_workspace_init")
 
 
 def workspace(device=None) -> torch.Tensor:
@@ -123,17 +137,22 @@ def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bo
             raise ValueError("teacher and student must share shape, strides and dtype")
         descs[r] = make_desc(xt, causal, scale, lengths)
         B, H, N, _ = xt.shape
+        if xt.device != dev or xs.device != dev:
+            raise ValueError("every relation must live on the same device")
         if out is not None:
             kl, st = out[r]
+            _check_out(kl, (B, H, N), "kl", dev)
+            _check_out(st, (B, H, N, 4), "stats", dev)
         else:
             kl = torch.empty((B, H, N), dtype=torch.float32, device=dev)
             st = torch.empty((B, H, N, 4), dtype=torch.float32, device=dev)
         outs.append((kl, st))
     ws = workspace(dev) if ws is None else ws
-    code = _abi.lib().relkl_fwd_qkv(
-        n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
-        _arr([_ptr(o[0]) for o in outs]), _arr([_ptr(o[1]) for o in outs]),
-        _ptr(ws), ws.numel(), _stream(dev, stream))
+    with torch.cuda.device(dev):
+        code = _abi.lib().relkl_fwd_qkv(
+            n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
+            _arr([_ptr(o[0]) for o in outs]), _arr([_ptr(o[1]) for o in outs]),
+            _ptr(ws), ws.numel(), _stream(dev, stream))
     check(code, "relkl_fwd_qkv")
     return outs
 
@@ -155,22 +174,23 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
         _cuda(xs, "x_s")
         if xt.shape != xs.shape or xt.stride() != xs.stride() or xt.dtype != xs.dtype:
             raise ValueError("teacher and student must share shape, strides and dtype")
+        if xt.device != dev or xs.device != dev:
+            raise ValueError("every relation must live on the same device")
         descs[r] = make_desc(xt, causal, scale, lengths)
-        if not stats[r].is_contiguous() or stats[r].dtype != torch.float32:
-            raise ValueError("stats must be contiguous float32 [B, H, N, 4]")
-        if dkl is not None and dkl[r] is not None and (not dkl[r].is_contiguous()
-                                                       or dkl[r].dtype != torch.float32):
-            raise ValueError("dkl must be contiguous float32 [B, H, N]")
+        B, H, N, _ = xt.shape
+        _check_out(stats[r], (B, H, N, 4), "stats", dev)
+        if dkl is not None and dkl[r] is not None:
+            _check_out(dkl[r], (B, H, N), "dkl", dev)
         dx = out[r] if out is not None else torch.empty(xs.shape, dtype=torch.float32, device=dev)
-        if not dx.is_contiguous() or dx.dtype != torch.float32:
-            raise ValueError("dx_s must be contiguous float32")
+        _check_out(dx, tuple(xs.shape), "dx_s", dev)
         dxs.append(dx)
     ws = workspace(dev) if ws is None else ws
     dkl_arr = None if dkl is None else _arr([_ptr(g) for g in dkl])
-    code = _abi.lib().relkl_bwd_qkv(
-        n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
-        _arr([_ptr(s) for s in stats]), dkl_arr, _arr([_ptr(d) for d in dxs]),
-        _ptr(ws), ws.numel(), _stream(dev, stream))
+    with torch.cuda.device(dev):
+        code = _abi.lib().relkl_bwd_qkv(
+            n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
+            _arr([_ptr(s) for s in stats]), dkl_arr, _arr([_ptr(d) for d in dxs]),
+            _ptr(ws), ws.numel(), _stream(dev, stream))
     check(code, "relkl_bwd_qkv")
     return dxs
 
@@ -179,7 +199,10 @@ def relkl_fwd(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True, scale: 
               kl: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
               ws: Optional[torch.Tensor] = None, stream=None,
               lengths: Optional[torch.Tensor] = None):
-    """Per-row KL [B,H,N] and statistics [B,H,N,4] of one relation."""
+    """Per-row KL [B,H,N] and statistics [B,H,N,4] of one relation.  Pass both
+    ``kl`` and ``stats`` to write into existing tensors, or neither."""
+    if (kl is None) != (stats is None):
+        raise ValueError("pass both kl and stats, or neither")
     out = None if kl is None else [(kl, stats)]
     return relkl_fwd_qkv([(x_t, x_s)], causal, scale, out=out, ws=ws, stream=stream,
                          lengths=lengths)[0]
@@ -210,14 +233,19 @@ def relkl_fwd_noalloc(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,
     _cuda(x_s, "x_s")
     if x_t.shape != x_s.shape or x_t.stride() != x_s.stride() or x_t.dtype != x_s.dtype:
         raise ValueError("teacher and student must share shape, strides and dtype")
+    if x_s.device != x_t.device:
+        raise ValueError("teacher and student must live on the same device")
     desc = make_desc(x_t, causal, scale, lengths)
     B, H, N, _ = x_t.shape
     if kl is None:
         kl = torch.empty((B, H, N), dtype=torch.float32, device=x_t.device)
     if stats is None:
         stats = torch.empty((B, H, N, 4), dtype=torch.float32, device=x_t.device)
-    code = _abi.lib().relkl_fwd_noalloc(ctypes.byref(desc), _ptr(x_t), _ptr(x_s), _ptr(kl),
-                                        _ptr(stats), _stream(x_t.device, stream))
+    _check_out(kl, (B, H, N), "kl", x_t.device)
+    _check_out(stats, (B, H, N, 4), "stats", x_t.device)
+    with torch.cuda.device(x_t.device):
+        code = _abi.lib().relkl_fwd_noalloc(ctypes.byref(desc), _ptr(x_t), _ptr(x_s), _ptr(kl),
+                                            _ptr(stats), _stream(x_t.device, stream))
     check(code, "relkl_fwd_noalloc")
     return kl, stats
 
@@ -226,8 +254,9 @@ def relkl_get_device_error(ws: Optional[torch.Tensor] = None, stream=None) -> Tu
     """Synchronise the stream and read the workspace record: (status, wait site)."""
     ws = workspace() if ws is None else ws
     where = ctypes.c_uint32(0)
-    code = _abi.lib().relkl_get_device_error(_ptr(ws), _stream(ws.device, stream),
-                                             ctypes.byref(where))
+    with torch.cuda.device(ws.device):
+        code = _abi.lib().relkl_get_device_error(_ptr(ws), _stream(ws.device, stream),
+                                                 ctypes.byref(where))
     return int(code), int(where.value)
 
 
@@ -275,10 +304,16 @@ def relkl_rope_bwd(dx_post: torch.Tensor, base: float, pos_scale: float = 1.0,
     B, H, N, d = (int(v) for v in dx_post.shape)
     if out is None:
         out = torch.empty(B, N, H, d, dtype=out_dtype, device=dx_post.device)
+    if (out.dtype != out_dtype or tuple(out.shape) != (B, N, H, d) or not out.is_contiguous()
+            or out.device != dx_post.device):
+        raise ValueError(f"out must be a contiguous {out_dtype} [B, N, H, d] tensor on "
+                         f"{dx_post.device}")
     rope = _abi.relkl_rope(float(base), float(pos_scale), float(pos_offset), 1 if apply else 0, 0)
-    check(_abi.lib().relkl_rope_bwd(B, H, N, d, _ptr(dx_post), ctypes.byref(rope),
-                                    _DTYPES[out_dtype], _ptr(out), _stream(dx_post.device, stream)),
-          "relkl_rope_bwd")
+    with torch.cuda.device(dx_post.device):
+        code = _abi.lib().relkl_rope_bwd(B, H, N, d, _ptr(dx_post), ctypes.byref(rope),
+                                         _DTYPES[out_dtype], _ptr(out),
+                                         _stream(dx_post.device, stream))
+    check(code, "relkl_rope_bwd")
     return out
 
 
@@ -296,10 +331,15 @@ def relkl_weight_grad(h: torch.Tensor, dx_pre: torch.Tensor, *, out: Optional[to
     cols = dx_pre.numel() // rows if rows else 0
     if rows * cols != dx_pre.numel():
         raise ValueError("h and dx_pre disagree on the number of token rows")
+    if dx_pre.device != h.device:
+        raise ValueError("h and dx_pre must live on the same device")
     if out is None:
         out = torch.empty(D, cols, dtype=torch.float32, device=h.device)
-    check(_abi.lib().relkl_weight_grad(rows, D, cols, _ptr(h), _ptr(dx_pre), _ptr(out),
-                                       _stream(h.device, stream)), "relkl_weight_grad")
+    _check_out(out, (D, cols), "dw", h.device)
+    with torch.cuda.device(h.device):
+        code = _abi.lib().relkl_weight_grad(rows, D, cols, _ptr(h), _ptr(dx_pre), _ptr(out),
+                                            _stream(h.device, stream))
+    check(code, "relkl_weight_grad")
     return out
 
 

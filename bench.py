@@ -35,6 +35,9 @@ import workload  # noqa: E402
 METRIC = "relation-KL fwd+bwd TFLOP/s & tokens/s at N=32K,d=128; % of BF16 tensor peak"
 L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's dense (no 2:4 sparsity) BF16 tensor-core figure for one B200: the
+# "% of dense BF16 tensor peak" of the metric is taken against this number.
+B200_DENSE_BF16_TFLOPS = 2250.0
 
 
 def flops(w: workload.Workload):
@@ -500,7 +503,17 @@ def main():
                        "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": f"inputs {in_bytes / 1e9:.2f} GB > L2 126 MB (no flush)"},
             "tokens_per_s": tokens,
-            "pct_bf16_peak": 100.0 * value / (peak_tf * world),
+            # the metric's "% of dense BF16 tensor peak": against the 2.25 PFLOP/s spec figure
+            "pct_bf16_peak": 100.0 * value / (B200_DENSE_BF16_TFLOPS * world),
+            # the same step against the measured cuBLAS bf16 GEMM rate (a plain library GEMM
+            # under the power cap: sustained figure, the clocks it ran at are listed below)
+            "pct_of_measured_cublas": 100.0 * value / (peak_tf * world),
+            "peak_reference": {
+                "spec_dense_bf16_tflops": B200_DENSE_BF16_TFLOPS,
+                "measured_bf16_tflops_sustained": peak_tf, "source": peak_src,
+                "measured_clocks": {k: v for k, v in peaks.items()
+                                    if "clock" in k or "mhz" in k.lower()},
+                "bench_sm_mhz_median": None},
             "fwd_ms": fwd_avg, "bwd_ms": bwd_avg,
             "fwd_tflops": fl_fwd / (fwd_avg * 1e-3) / 1e12,
             "bwd_tflops": fl_bwd / (bwd_avg * 1e-3) / 1e12,
@@ -525,6 +538,7 @@ def main():
             "input_generation_s": t_gen,
             "cpu_baseline": cpu,
         }
+        result["peak_reference"]["bench_sm_mhz_median"] = clk.get("sm_mhz")
         print(json.dumps(result), flush=True)
     if world > 1:
         dist.barrier()

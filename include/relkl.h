@@ -108,8 +108,11 @@ relkl_status relkl_fwd(const relkl_desc* desc, const void* x_t, const void* x_s,
  *   dkl      : float [B, H, N] contiguous upstream gradient of kl, or NULL for
  *              1/N on every row (the gradient of L = (1/N) sum_i kl_i).
  *   dx_s     : float [B, H, N, d] contiguous, out: overwritten with dL/dX_s.
- * The teacher is frozen and gets no gradient.  dx_s is accumulated with
- * float32 atomics, so its last bits depend on scheduling.                   */
+ * The teacher is frozen and gets no gradient.  dx_s is zeroed on `stream`
+ * and then accumulated by float32 reduce-adds performed in L2 (TMA bulk-tensor
+ * reductions on the tensor-core path, atomics on the CUDA-core path); the
+ * order of those additions depends on scheduling, so the last bits of dx_s
+ * may differ between runs.                                                  */
 relkl_status relkl_bwd(const relkl_desc* desc, const void* x_t, const void* x_s,
                        const float* stats, const float* dkl, float* dx_s,
                        void* ws, size_t ws_bytes, void* stream);
@@ -165,8 +168,11 @@ int32_t relkl_path_for(const relkl_desc* desc);
  * (relkl_workspace_bytes()) exceeded that size would be refused with
  * RELKL_ERR_WORKSPACE; the need does not grow with B, H or N.
  *  - The first call on a device looks up the array's device address (with
- *    that device current) and keeps it; make that first call before any
- *    stream capture.
+ *    that device current) and keeps it together with the device's current
+ *    context; make that first call before any stream capture.  A later call
+ *    that finds another context current on the device (after cudaDeviceReset,
+ *    for example) looks the address up again.
+ *  - The current device must be the one that owns the tensors and `stream`.
  *  - All calls share the one array, which keeps what the last call wrote;
  *    each call clears the record on its stream before its kernel starts.
  *    Calls that overlap on the GPU (other streams, other threads) race on the

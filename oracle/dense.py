@@ -46,7 +46,7 @@ import numpy as np
 import torch
 
 __all__ = ["as_f64", "relation_logits", "allowed", "fwd_unit", "bwd_unit",
-           "fwd_rows", "bwd_rows", "fwd", "bwd", "unit_loss"]
+           "fwd_rows", "bwd_rows", "fwd", "bwd", "unit_loss", "relation_probs"]
 
 
 def as_f64(x) -> np.ndarray:
@@ -230,3 +230,16 @@ def unit_loss(kl_rows: np.ndarray) -> float:
     """L = (1/n) sum_i kl_i for one unit's rows."""
     kl_rows = np.asarray(kl_rows, dtype=np.float64)
     return float(kl_rows.sum() / kl_rows.shape[-1])
+
+
+def relation_probs(xt, xs, causal: bool = True, scale: Optional[float] = None):
+    """Dense row distributions (R_t, R_s) of one small unit, zero on masked
+    entries.  For tests that need the whole matrices (e.g. rounding-error
+    bounds); the product path never forms them."""
+    xt, xs = as_f64(xt), as_f64(xs)
+    N, d = xt.shape
+    s = _scale(d, scale)
+    ok = allowed(np.arange(N), N, causal)
+    logp_t, _, _ = _masked_log_softmax(relation_logits(xt, xt, s), ok)
+    logp_s, _, _ = _masked_log_softmax(relation_logits(xs, xs, s), ok)
+    return np.where(ok, np.exp(logp_t), 0.0), np.where(ok, np.exp(logp_s), 0.0)

@@ -162,3 +162,20 @@ def test_weight_grad_validation():
         (8, 64, 64, p, None, p), (8, 64, 64, p, p, None), (8, 64, 64, ctypes.c_void_p(4104), p, p),
     ]:
         assert lib.relkl_weight_grad(rows, D, cols, h, dx, dw, None) == inv
+
+
+def test_binding_rejects_bad_outputs_before_the_call():
+    """The binding checks caller-provided outputs (shape, dtype, contiguity,
+    device) before handing raw pointers to the library, which writes B*H*N
+    floats of kl and B*H*N*4 of stats through them."""
+    import torch
+    from attention_relation_kl_b200.ops import _check_out
+    dev = torch.device("cpu")
+    ok = torch.empty(2, 3, 5, dtype=torch.float32)
+    _check_out(ok, (2, 3, 5), "kl", dev)
+    for bad in (torch.empty(2, 3, 4), torch.empty(2, 3, 5, dtype=torch.float64),
+                torch.empty(2, 5, 3).transpose(1, 2), torch.empty(2, 3, 5, device="meta")):
+        with pytest.raises(ValueError):
+            _check_out(bad, (2, 3, 5), "kl", dev)
+    with pytest.raises(ValueError):
+        _check_out(None, (2, 3, 5), "kl", dev)

@@ -12,7 +12,9 @@ import torch
 import attention_relation_kl_b200 as rk
 import workload
 from oracle import dense
-from parity import DX_TOL_BF16, DX_TOL_FP32, assert_dx, assert_kl, assert_stats, to_np
+from parity import DX_TOL_BF16, assert_dx, assert_kl, assert_stats, fp32_dx_tolerance, to_np
+
+FP32 = "fp32"   # dx_tol marker: derive the fp32-path tolerance from the input
 
 pytestmark = pytest.mark.gpu
 
@@ -29,20 +31,25 @@ def _device_ok():
     assert code == 0, f"device wait ran out at site {where}"
 
 
-def check_full(xt, xs, causal=True, dkl=None, dx_tol=DX_TOL_BF16, path=None):
-    """Run fwd+bwd on the GPU and compare every output with the oracle."""
+def check_full(xt, xs, causal=True, dkl=None, dx_tol=DX_TOL_BF16, path=None, scale=0.0):
+    """Run fwd+bwd on the GPU and compare every output with the oracle.
+    ``scale`` is the desc's logit scale (0: 1/sqrt(d)); dx_tol=FP32 derives
+    the fp32-path tolerance from the input's own arithmetic."""
     dev = "cuda"
     gt, gs = xt.to(dev), xs.to(dev)
     if path is not None:
-        assert rk.relkl_path_for(gt, causal) == path
-    kl, st = rk.relkl_fwd(gt, gs, causal)
-    dx = rk.relkl_bwd(gt, gs, st, None if dkl is None else dkl.to(dev), causal)
+        assert rk.relkl_path_for(gt, causal, scale) == path
+    kl, st = rk.relkl_fwd(gt, gs, causal, scale)
+    dx = rk.relkl_bwd(gt, gs, st, None if dkl is None else dkl.to(dev), causal, scale)
     torch.cuda.synchronize()
     _device_ok()
-    ref = dense.fwd(xt, xs, causal)
+    oscale = scale if scale else None
+    ref = dense.fwd(xt, xs, causal, oscale)
     assert_kl(to_np(kl), ref["kl"])
     assert_stats(to_np(st), ref)
-    assert_dx(to_np(dx), dense.bwd(xt, xs, dkl, causal), dx_tol)
+    if dx_tol == FP32:
+        dx_tol = fp32_dx_tolerance(xt, xs, dkl, causal, oscale)
+    assert_dx(to_np(dx), dense.bwd(xt, xs, dkl, causal, oscale), dx_tol)
 
 
 def q_inputs(B, H, N, d, dtype="bf16", seed=0, causal=True, pi=4.0):
@@ -93,15 +100,51 @@ def test_tc_value_relation_small_kl():
     check_full(xt, xs)
 
 
+# ------------------------------------------------- explicit logit scale
+# The desc's scale replaces 1/sqrt(d) everywhere: in the logits, the LSEs and
+# the factor s of dX = s (G + G^T) X_s.  Every kernel family, both masks.
+@pytest.mark.parametrize("N,d,scale,causal,path", [
+    (700, 128, 0.05, True, 1), (700, 128, 0.3, False, 1),      # one-block backward
+    (4200, 128, 0.05, False, 1), (4200, 128, 0.3, True, 1),    # paired-block backward
+    (513, 64, 0.05, True, 1), (513, 64, 0.3, False, 1),        # d = 64
+    (150, 64, 0.05, True, 2), (150, 64, 0.3, False, 2),        # CUDA-core fp32
+])
+def test_explicit_scale(N, d, scale, causal, path):
+    dtype = "bf16" if path == 1 else "fp32"
+    xt, xs = q_inputs(1, 2 if N < 1000 else 1, N, d, dtype=dtype, seed=N + int(1000 * scale),
+                      causal=causal)
+    check_full(xt, xs, causal=causal, path=path, scale=scale,
+               dx_tol=DX_TOL_BF16 if path == 1 else FP32)
+
+
+# ------------------------------------------------- large logits
+# Rows clustered around a few shared directions: logits reach ~70-100 across
+# whole clusters (not only on the diagonal), so the shared running maximum
+# moves by tens between tiles, most exponentials underflow and the KL stays
+# of order 0.3.  Both masks, both backwards at d = 128, d = 64 and fp32.
+@pytest.mark.parametrize("N,d,causal,dtype", [
+    (4200, 128, True, "bf16"), (4200, 128, False, "bf16"), (1000, 128, True, "bf16"),
+    (700, 64, False, "bf16"), (4300, 64, True, "bf16"), (200, 64, True, "fp32"),
+])
+def test_large_logits(N, d, causal, dtype):
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    xt, xs = workload.clustered_pair((1, 1, N, d), seed=N + d, amplitude=2.5 if d == 128 else 3.0,
+                                     dtype=tdt)
+    ref_m = dense.fwd_rows(xt[0, 0], xs[0, 0], range(0, N, 97), causal)["m"]
+    assert ref_m.max() > 60.0     # the case really has large logits
+    check_full(xt, xs, causal=causal, path=1 if dtype == "bf16" else 2,
+               dx_tol=DX_TOL_BF16 if dtype == "bf16" else FP32)
+
+
 def test_simt_fp32_tiny_config():
     w = workload.CONFIGS["tiny_fp32_n256"]
     xt, xs = workload.generate(w)["q"]
-    check_full(xt, xs, dx_tol=DX_TOL_FP32, path=2)
+    check_full(xt, xs, dx_tol=FP32, path=2)
 
 
 def test_simt_bf16_unsupported_head_dim():
     xt, xs = q_inputs(1, 2, 200, 96, seed=3)
-    check_full(xt, xs, dx_tol=DX_TOL_FP32, path=2)
+    check_full(xt, xs, dx_tol=FP32, path=2)
 
 
 def test_upstream_gradient():
@@ -109,7 +152,7 @@ def test_upstream_gradient():
     dkl = torch.randn(2, 2, 260, generator=torch.Generator().manual_seed(2)) / 260
     check_full(xt, xs, dkl=dkl)
     xt32, xs32 = q_inputs(1, 1, 70, 64, dtype="fp32", seed=12)
-    check_full(xt32, xs32, dkl=torch.linspace(-1, 1, 70).reshape(1, 1, 70), dx_tol=DX_TOL_FP32)
+    check_full(xt32, xs32, dkl=torch.linspace(-1, 1, 70).reshape(1, 1, 70), dx_tol=FP32)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
@@ -179,6 +222,27 @@ def test_forward_is_deterministic():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+def test_binding_rejects_wrong_outputs():
+    xt, xs = q_inputs(1, 2, 200, 128, seed=19)
+    gt, gs = xt.cuda(), xs.cuda()
+    good_kl = torch.empty(1, 2, 200, device="cuda")
+    good_st = torch.empty(1, 2, 200, 4, device="cuda")
+    with pytest.raises(ValueError):
+        rk.relkl_fwd(gt, gs, kl=torch.empty(1, 2, 199, device="cuda"), stats=good_st)
+    with pytest.raises(ValueError):
+        rk.relkl_fwd(gt, gs, kl=good_kl, stats=torch.empty(1, 2, 200, 3, device="cuda"))
+    with pytest.raises(ValueError):
+        rk.relkl_fwd(gt, gs, kl=good_kl)                       # stats missing
+    with pytest.raises(ValueError):
+        rk.relkl_fwd_noalloc(gt, gs, kl=good_kl.double(), stats=good_st)
+    with pytest.raises(ValueError):
+        rk.relkl_fwd_noalloc(gt, gs, kl=good_kl, stats=good_st.transpose(0, 1))
+    kl, st = rk.relkl_fwd(gt, gs, kl=good_kl, stats=good_st)
+    with pytest.raises(ValueError):
+        rk.relkl_bwd(gt, gs, st, dx_s=torch.empty(1, 2, 200, 128, device="cuda").half())
+    torch.cuda.synchronize()
+
+
 def test_autograd_wrapper():
     xt, xs = q_inputs(1, 2, 200, 128, seed=17)
     gt = xt.cuda()
@@ -196,7 +260,35 @@ def test_autograd_wrapper():
 SAMPLE_ROWS = (0, 1, 127, 128, 129)
 
 
-def _sampled(w: workload.Workload, units, dx_units, n_dx_rows=6):
+def _dx_rows(N):
+    """Rows whose dX is compared at workload size: first, second, middle and last
+    rows of the 128-row blocks that the first, a middle and the last work item
+    of the paired-block backward hold (blocks 2k and 2k+1 of its two pair
+    sequences k = npb-1-m and k = m), plus the unit's last two rows."""
+    nblk = (N + 127) // 128
+    npb = (nblk + 1) // 2
+    items = (npb + 1) // 2
+    blocks = set()
+    for m in sorted({0, items // 2, items - 1}):
+        for k in (npb - 1 - m, m):
+            blocks.update(b for b in (2 * k, 2 * k + 1) if 0 <= b < nblk)
+    rows = set()
+    for b in blocks:
+        r0 = b * 128
+        rows.update(r for r in (r0, r0 + 1, r0 + 63, r0 + 64, r0 + 126, r0 + 127) if r < N)
+    rows.update(r for r in (N - 2, N - 1) if r >= 0)
+    return sorted(rows)
+
+
+def test_dx_rows_cover_pair_items():
+    rows = _dx_rows(32768)
+    assert len(rows) >= 64
+    blocks = {r // 128 for r in rows}
+    # first item: pairs 127 and 0; middle (m = 32): 95 and 32; last (m = 63): 64 and 63
+    assert blocks == {254, 255, 0, 1, 190, 191, 64, 65, 128, 129, 126, 127}
+
+
+def _sampled(w: workload.Workload, units, dx_units):
     """Fused Q/K/V launch of the whole workload; oracle on sampled units."""
     x = workload.generate(w)
     pairs = [(x[r][0].cuda(), x[r][1].cuda()) for r in w.relations]
@@ -218,7 +310,7 @@ def _sampled(w: workload.Workload, units, dx_units, n_dx_rows=6):
         assert_kl(to_np(kl[b, h])[sel], ref["kl"], what=f"kl[{rel},{b},{h}]")
         assert_stats(to_np(st[b, h])[sel], ref)
         if full:
-            dx_rows = rows[:n_dx_rows] + rows[-2:]
+            dx_rows = _dx_rows(N)
             ref_dx = dense.bwd_rows(xt, xs, dx_rows, causal=w.causal, lse=ref)
             got = to_np(dxs[rel_idx[rel]][b, h])[dx_rows]
             assert_dx(got, ref_dx, DX_TOL_BF16)
@@ -233,20 +325,28 @@ def test_config_llama2_h32_n4k():
 def test_config_gqa_llama3_n16k():
     w = workload.CONFIGS["gqa_llama3_n16k"]
     units = [("q", 1, 31), ("k", 0, 3), ("v", 1, 7)]
-    _sampled(w, units, dx_units={("v", 1, 7)})
+    _sampled(w, units, dx_units=set(units))
 
 
 def test_config_ext_h32_n32k():
     w = workload.CONFIGS["ext_h32_n32k"]
     units = [("q", 0, 0), ("k", 0, 17), ("v", 0, 31)]
-    _sampled(w, units, dx_units={("q", 0, 0)})
+    _sampled(w, units, dx_units=set(units))
+
+
+def test_config_d64_h32_n32k():
+    # head dimension 64 at the 32K shape: kl on every row and dX on the
+    # sampled rows of one unit of each relation
+    w = workload.CONFIGS["d64_h32_n32k"]
+    units = [("q", 0, 0), ("k", 0, 17), ("v", 0, 31)]
+    _sampled(w, units, dx_units=set(units))
 
 
 def test_config_sweep_n64k():
     # the largest point of the sequence-length sweep: B=1, H=32, N=65536
     w = workload.sweep_config(65536)
     units = [("q", 0, 0), ("k", 0, 9), ("v", 0, 31)]
-    _sampled(w, units, dx_units={("k", 0, 9)})
+    _sampled(w, units, dx_units=set(units))
 
 
 # ------------------------------------------------------ right padding
@@ -285,7 +385,7 @@ def test_padded_lengths(B, H, N, d, dtype, causal, lengths, path):
         assert np.all(to_np(kl[b, :, L:]) == 0) and np.all(to_np(st[b, :, L:]) == 0)
         if L:
             assert_stats(to_np(st[b, :, :L]), {k: v[b, :, :L] for k, v in ref.items()})
-    tol = DX_TOL_BF16 if path == 1 else DX_TOL_FP32
+    tol = DX_TOL_BF16 if path == 1 else fp32_dx_tolerance(xt, xs, None, causal, lengths=lengths)
     ref_dx = dense.bwd(xt, xs, None, causal, lengths=lengths)
     assert_dx(to_np(dx), ref_dx, tol)
     for b, L in enumerate(lengths):

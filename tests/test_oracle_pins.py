@@ -100,6 +100,31 @@ def test_uniform_vs_onehot_golden():
             G[i, j] = dkl[i] * (rs - 1.0 / (i + 1))
     dx_ref = s * c * (G + G.T)
     np.testing.assert_allclose(dense.bwd_unit(xt, xs, dkl=dkl), dx_ref, rtol=1e-12, atol=1e-16)
+    # the unit loss L = (1/n) sum_i kl_i of the same closed form
+    L_ref = sum(kl_ref) / N
+    assert abs(dense.unit_loss(r["kl"]) - L_ref) <= 1e-14 * abs(L_ref)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_unit_loss_matches_default_backward(causal):
+    """L = (1/n) sum_i kl_i is the loss whose gradient the default upstream
+    gradient (1/n per row) produces: central differences of unit_loss with
+    respect to X_s equal bwd_unit(dkl=None).  A wrong normaliser (sum, 1/(n-1))
+    or a wrong row count fails this."""
+    N, d = 9, 4
+    xt, xs = _rand_pair(N, d, seed=77)
+    g = dense.bwd_unit(xt, xs, None, causal)
+    h = 1e-6
+    fd = np.zeros_like(xs)
+    for i in range(N):
+        for k in range(d):
+            xp, xm = xs.copy(), xs.copy()
+            xp[i, k] += h
+            xm[i, k] -= h
+            lp = dense.unit_loss(dense.fwd_unit(xt, xp, causal)["kl"])
+            lm = dense.unit_loss(dense.fwd_unit(xt, xm, causal)["kl"])
+            fd[i, k] = (lp - lm) / (2 * h)
+    np.testing.assert_allclose(fd, g, rtol=1e-6, atol=1e-10)
 
 
 # ------------------------------------------------------- library cross-check

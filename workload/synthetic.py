@@ -33,7 +33,7 @@ from typing import Dict, Optional, Tuple
 import torch
 
 __all__ = ["Workload", "CONFIGS", "get_config", "sweep_config", "generate",
-           "rope_rotate", "unit_list"]
+           "rope_rotate", "unit_list", "clustered_pair"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -188,4 +188,29 @@ def gaussian_pair(shape, seed: int, noise: float, dtype: torch.dtype = torch.flo
     gen = torch.Generator().manual_seed(seed)
     xt = _draw(gen, shape)
     xs = xt.to(torch.float64) + noise * _draw(gen, shape).to(torch.float64)
+    return xt.to(dtype).contiguous(), xs.to(dtype).contiguous()
+
+
+def clustered_pair(shape, seed: int, n_clusters: int = 4, amplitude: float = 2.5,
+                   spread: float = 0.5, student_noise: float = 0.3,
+                   dtype: torch.dtype = torch.bfloat16):
+    """Rows drawn around a few shared directions, for logits far larger than
+    unit-variance activations give.
+
+    Draw order: cluster centres c ~ N(0,1) [n_clusters, d], the cluster of each
+    row (uniform), the teacher's spread eps ~ N(0,1), the student's noise
+    eta ~ N(0,1).  x_t = amplitude * c[k(row)] + spread * eps and
+    x_s = x_t + student_noise * eta.  Rows of one cluster share a large common
+    component, so with the 1/sqrt(d) scale their mutual logits sit near
+    amplitude^2 sqrt(d) (about 70 for amplitude 2.5 and d = 128) rather than on
+    the diagonal alone, and each row's distribution spreads over its cluster.
+    """
+    *lead, n, d = shape
+    gen = torch.Generator().manual_seed(seed)
+    centres = _draw(gen, (n_clusters, d)).to(torch.float64)
+    which = torch.randint(0, n_clusters, tuple(lead) + (n,), generator=gen)
+    eps = _draw(gen, shape).to(torch.float64)
+    eta = _draw(gen, shape).to(torch.float64)
+    xt = amplitude * centres[which] + spread * eps
+    xs = xt + student_noise * eta
     return xt.to(dtype).contiguous(), xs.to(dtype).contiguous()
