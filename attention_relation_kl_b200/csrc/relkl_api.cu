@@ -216,7 +216,8 @@ bool use_tc(int32_t n_rel, const relkl_desc* descs, const void* const* xt, const
 }
 
 relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const* xt,
-                      const void* const* xs, TcParams* p, void* ws) {
+                      const void* const* xs, TcParams* p, void* ws, int part = 0,
+                      int n_parts = 1) {
   std::memset(p, 0, sizeof(*p));
   const relkl_desc& d0 = descs[0];
   int seg = 0, ub = 0;
@@ -237,7 +238,11 @@ relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const*
   p->N = d0.N;
   p->nblk = (d0.N + 127) / 128;
   p->n_pairs = (p->nblk + 1) / 2;
-  p->n_items = ub * p->n_pairs;
+  p->n_units = ub;
+  p->part = part;
+  p->n_parts = n_parts;
+  p->n_local = part < p->n_pairs ? (p->n_pairs - part + n_parts - 1) / n_parts : 0;
+  p->n_items = ub * p->n_local;
   p->causal = d0.causal;
   p->scale = logit_scale(d0);
   p->sl2 = p->scale * 1.4426950408889634f;
@@ -247,7 +252,7 @@ relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const*
 }
 
 relkl_status build_simt(int32_t n_rel, const relkl_desc* descs, const void* const* xt,
-                        const void* const* xs, SimtParams* p) {
+                        const void* const* xs, SimtParams* p, int part = 0, int n_parts = 1) {
   std::memset(p, 0, sizeof(*p));
   const relkl_desc& d0 = descs[0];
   int seg = 0, ub = 0;
@@ -273,6 +278,10 @@ relkl_status build_simt(int32_t n_rel, const relkl_desc* descs, const void* cons
   p->is_bf16 = d0.dtype == RELKL_BF16;
   p->scale = logit_scale(d0);
   p->n_units = ub;
+  p->part = part;
+  p->n_parts = n_parts;
+  const int nblk32 = (d0.N + 31) / 32;
+  p->nblk_local = part < nblk32 ? (nblk32 - part + n_parts - 1) / n_parts : 0;
   return RELKL_OK;
 }
 
@@ -311,10 +320,14 @@ int32_t relkl_path_for(const relkl_desc* desc) {
   return tc_shape(*desc) ? 1 : 2;
 }
 
-relkl_status relkl_fwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
-                           const void* const* x_s, float* const* kl, float* const* stats,
-                           void* ws, size_t ws_bytes, void* stream) {
-  NvtxRange nvtx_range("relkl_fwd_qkv");
+}  // extern "C"
+
+namespace {
+
+relkl_status fwd_impl(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
+                      const void* const* x_s, float* const* kl, float* const* stats, int32_t part,
+                      int32_t n_parts, void* ws, size_t ws_bytes, void* stream) {
+  if (n_parts < 1 || part < 0 || part >= n_parts) return RELKL_ERR_INVALID;
   bool empty = false;
   relkl_status s = check_multi(n_rel, descs, x_t, x_s, &empty);
   if (s != RELKL_OK || empty) return s;
@@ -330,24 +343,25 @@ relkl_status relkl_fwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* c
   cudaError_t e;
   if (use_tc(n_rel, descs, x_t, x_s)) {
     TcParams p;
-    if ((s = build_tc(n_rel, descs, x_t, x_s, &p, ws)) != RELKL_OK) return s;
+    if ((s = build_tc(n_rel, descs, x_t, x_s, &p, ws, part, n_parts)) != RELKL_OK) return s;
     set_seg_outputs(&p, n_rel, descs, kl, stats, nullptr, nullptr, nullptr);
+    if (p.n_items == 0) return RELKL_OK;   // this part holds no work item
     const int grid = p.n_items < dev.sms ? p.n_items : dev.sms;
     e = tc_launch_fwd(p, descs[0].d, grid, st);
   } else {
     SimtParams p;
-    build_simt(n_rel, descs, x_t, x_s, &p);
+    build_simt(n_rel, descs, x_t, x_s, &p, part, n_parts);
     set_seg_outputs(&p, n_rel, descs, kl, stats, nullptr, nullptr, nullptr);
     e = simt_launch_fwd(p, st);
   }
   return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
 }
 
-relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
-                           const void* const* x_s, const float* const* stats,
-                           const float* const* dkl, float* const* dx_s, void* ws,
-                           size_t ws_bytes, void* stream) {
-  NvtxRange nvtx_range("relkl_bwd_qkv");
+relkl_status bwd_impl(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
+                      const void* const* x_s, const float* const* stats, const float* const* dkl,
+                      float* const* dx_s, int32_t part, int32_t n_parts, void* ws,
+                      size_t ws_bytes, void* stream) {
+  if (n_parts < 1 || part < 0 || part >= n_parts) return RELKL_ERR_INVALID;
   bool empty = false;
   relkl_status s = check_multi(n_rel, descs, x_t, x_s, &empty);
   if (s != RELKL_OK || empty) return s;
@@ -368,7 +382,7 @@ relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* c
   TcParams tp;
   SimtParams sp;
   if (tc) {
-    if ((s = build_tc(n_rel, descs, x_t, x_s, &tp, ws)) != RELKL_OK) return s;
+    if ((s = build_tc(n_rel, descs, x_t, x_s, &tp, ws, part, n_parts)) != RELKL_OK) return s;
     set_seg_outputs(&tp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);
     for (int r = 0, seg = 0; r < n_rel; ++r) {
       if (!n_units(descs[r])) continue;
@@ -379,7 +393,7 @@ relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* c
       if ((s = encode_x(&sg.tm_s64, descs[r], x_s[r], 64)) != RELKL_OK) return s;
     }
   } else {
-    build_simt(n_rel, descs, x_t, x_s, &sp);
+    build_simt(n_rel, descs, x_t, x_s, &sp, part, n_parts);
     set_seg_outputs(&sp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);
   }
   // dX_s is accumulated with atomics: clear it first (same stream)
@@ -389,12 +403,48 @@ relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* c
     if ((e = launch_zero(dx_s[r], n, dev.sms, st)) != cudaSuccess) return cuda_fail(e);
   }
   if (tc) {
-    const int grid = tp.n_items < dev.sms ? tp.n_items : dev.sms;
-    e = tc_launch_bwd(tp, descs[0].d, grid, st);
+    // the launcher sizes the grid (at most one CTA per SM) from the work items
+    // of the kernel it picks; a part without items launches nothing
+    e = tc_launch_bwd(tp, descs[0].d, dev.sms, st);
   } else {
     e = simt_launch_bwd(sp, st);
   }
   return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+relkl_status relkl_fwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
+                           const void* const* x_s, float* const* kl, float* const* stats,
+                           void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("relkl_fwd_qkv");
+  return fwd_impl(n_rel, descs, x_t, x_s, kl, stats, 0, 1, ws, ws_bytes, stream);
+}
+
+relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
+                           const void* const* x_s, const float* const* stats,
+                           const float* const* dkl, float* const* dx_s, void* ws,
+                           size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("relkl_bwd_qkv");
+  return bwd_impl(n_rel, descs, x_t, x_s, stats, dkl, dx_s, 0, 1, ws, ws_bytes, stream);
+}
+
+relkl_status relkl_fwd_qkv_part(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
+                                const void* const* x_s, float* const* kl, float* const* stats,
+                                int32_t part, int32_t n_parts, void* ws, size_t ws_bytes,
+                                void* stream) {
+  NvtxRange nvtx_range("relkl_fwd_qkv_part");
+  return fwd_impl(n_rel, descs, x_t, x_s, kl, stats, part, n_parts, ws, ws_bytes, stream);
+}
+
+relkl_status relkl_bwd_qkv_part(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
+                                const void* const* x_s, const float* const* stats,
+                                const float* const* dkl, float* const* dx_s, int32_t part,
+                                int32_t n_parts, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("relkl_bwd_qkv_part");
+  return bwd_impl(n_rel, descs, x_t, x_s, stats, dkl, dx_s, part, n_parts, ws, ws_bytes, stream);
 }
 
 relkl_status relkl_fwd(const relkl_desc* desc, const void* x_t, const void* x_s, float* kl,

@@ -33,8 +33,13 @@ struct TcParams {
   int n_seg;
   int N;
   int nblk;       // ceil(N / 128)
-  int n_pairs;    // ceil(nblk / 2): row blocks p and nblk-1-p form one work item
-  int n_items;    // units * n_pairs
+  int n_pairs;    // work items per unit (forward: ceil(nblk / 2), row blocks p and nblk-1-p)
+  int n_units;
+  // A call may cover one part of every unit's work items: items
+  // part, part + n_parts, ... (rows of the other parts are not touched).
+  int part, n_parts;
+  int n_local;    // items per unit in this part: ceil((n_pairs - part) / n_parts)
+  int n_items;    // n_units * n_local
   int causal;
   float scale;    // logit scale
   float sl2;      // scale * log2(e)
@@ -65,6 +70,8 @@ struct SimtParams {
   int is_bf16;
   float scale;
   int n_units;
+  int part, n_parts;   // 32-row blocks part, part + n_parts, ... of every unit
+  int nblk_local;      // ceil((ceil(N / 32) - part) / n_parts)
 };
 
 }  // namespace relkl

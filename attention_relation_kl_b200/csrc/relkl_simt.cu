@@ -65,7 +65,9 @@ relkl_fwd_simt_kernel(const __grid_constant__ SimtParams p) {
   float* xsj = xtj + SB * pitch;
 
   const int nblk = (p.N + SB - 1) / SB;
-  const int u = blockIdx.x / nblk, I = blockIdx.x - (blockIdx.x / nblk) * nblk;
+  // this call's 32-row blocks of the unit: part, part + n_parts, ...
+  const int u = blockIdx.x / p.nblk_local;
+  const int I = p.part + (blockIdx.x - u * p.nblk_local) * p.n_parts;
   const SimtUnit U = simt_unit(p, u);
   const SimtSeg& S = *U.seg;
   const int rr = threadIdx.x >> 3, cg = threadIdx.x & 7;
@@ -147,7 +149,9 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
   float* g = xsj + SB * pitch;      // [32][33]
 
   const int nblk = (p.N + SB - 1) / SB;
-  const int u = blockIdx.x / nblk, I = blockIdx.x - (blockIdx.x / nblk) * nblk;
+  // this call's 32-row blocks of the unit: part, part + n_parts, ...
+  const int u = blockIdx.x / p.nblk_local;
+  const int I = p.part + (blockIdx.x - u * p.nblk_local) * p.n_parts;
   const SimtUnit U = simt_unit(p, u);
   const SimtSeg& S = *U.seg;
   const int rr = threadIdx.x >> 3, cg = threadIdx.x & 7;
@@ -234,24 +238,24 @@ static size_t simt_smem(int d, int bwd) {
 }
 
 cudaError_t simt_launch_fwd(const SimtParams& p, cudaStream_t stream) {
-  const int nblk = (p.N + SB - 1) / SB;
+  if (p.n_units * p.nblk_local == 0) return cudaSuccess;
   const size_t sm = simt_smem(p.d, 0);
   cudaError_t e = cudaFuncSetAttribute(relkl_fwd_simt_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sm));
   if (e != cudaSuccess) return e;
-  relkl_fwd_simt_kernel<<<p.n_units * nblk, SIMT_THREADS, sm, stream>>>(p);
+  relkl_fwd_simt_kernel<<<p.n_units * p.nblk_local, SIMT_THREADS, sm, stream>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t simt_launch_bwd(const SimtParams& p, cudaStream_t stream) {
-  const int nblk = (p.N + SB - 1) / SB;
+  if (p.n_units * p.nblk_local == 0) return cudaSuccess;
   const size_t sm = simt_smem(p.d, 1);
   cudaError_t e = cudaFuncSetAttribute(relkl_bwd_simt_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sm));
   if (e != cudaSuccess) return e;
-  relkl_bwd_simt_kernel<<<p.n_units * nblk, SIMT_THREADS, sm, stream>>>(p);
+  relkl_bwd_simt_kernel<<<p.n_units * p.nblk_local, SIMT_THREADS, sm, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -72,6 +72,13 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
   return out;
 }
 
+// Work item -> (unit u, per-unit item index pp).  A call that covers one part
+// of the work takes the unit's items part, part + n_parts, ...
+__device__ __forceinline__ void decode_item(const TcParams& p, int item, int& u, int& pp) {
+  u = item / p.n_local;
+  pp = p.part + (item - u * p.n_local) * p.n_parts;
+}
+
 // Row blocks of one work item: pass 0 is the longer block nblk-1-p, pass 1
 // (absent when both coincide) is block p.
 // Valid rows and columns of unit U: its batch element's length, or all N.
@@ -200,7 +207,8 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
       uint32_t nI = 0, nJ = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        int u, pp;
+        decode_item(p, item, u, pp);
         const Unit U = decode_unit(p, u);
         for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
           const int I = pass_block(p, pp, pass);
@@ -248,7 +256,8 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
       const uint32_t dXsI = sw128_desc_lo(base + L::XS_I, 16);
       const uint32_t ring0 = sw128_desc_lo(base + L::RING, 16);
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        int u, pp;
+        decode_item(p, item, u, pp);
         (void)u;
         for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
           const int I = pass_block(p, pp, pass);
@@ -290,7 +299,8 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
     uint32_t nt = 0, nm = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      int u, pp;
+        decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
       for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
         const int I = pass_block(p, pp, pass);
@@ -582,7 +592,8 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       uint32_t armsS[2] = {0, 0};   // loads issued per ring stage
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        int u, pp;
+        decode_item(p, item, u, pp);
         const Unit U = decode_unit(p, u);
         for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
           const int I = pass_block(p, pp, pass);
@@ -661,7 +672,8 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
         return true;
       };
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        int u, pp;
+        decode_item(p, item, u, pp);
         (void)u;
         for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
           const int I = pass_block(p, pp, pass);
@@ -707,7 +719,8 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
     uint32_t np = 0, nrb = 0, nstg = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      int u, pp;
+        decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
       for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
         const int I = pass_block(p, pp, pass);
@@ -744,7 +757,8 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
     uint32_t ns = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      int u, pp;
+        decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
       for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
         const int I = pass_block(p, pp, pass);
@@ -937,7 +951,8 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
       uint32_t armsT[2] = {0, 0}, armsS[4] = {0, 0, 0, 0};
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        int u, pp;
+        decode_item(p, item, u, pp);
         const Unit U = decode_unit(p, u);
         for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
           const int I = pass_block(p, pp, pass);
@@ -1029,7 +1044,8 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
         return true;
       };
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+        int u, pp;
+        decode_item(p, item, u, pp);
         (void)u;
         for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
           const int I = pass_block(p, pp, pass);
@@ -1087,7 +1103,8 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
     uint32_t np = 0, nrb = 0, nstg = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      int u, pp;
+        decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
       for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
         const int I = pass_block(p, pp, pass);
@@ -1151,7 +1168,8 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
     uint32_t ns = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int u = item / p.n_pairs, pp = item - u * p.n_pairs;
+      int u, pp;
+        decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
       for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
         const int I = pass_block(p, pp, pass);
@@ -1348,7 +1366,6 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int ipu = p.n_pairs;   // pair items per unit
 
   if (warp == BWD_TMA_WARP) {
     // ------------------------------------------------------------ TMA
@@ -1364,7 +1381,8 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
       uint32_t armsT[2] = {0, 0}, armsS[2] = {0, 0};
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int u = item / ipu, m = item - u * ipu;
+        int u, m;
+        decode_item(p, item, u, m);
         const Unit U = decode_unit(p, u);
         for (int w = 0; ok && w < 2; ++w) {
           const int R0 = pair_seq_block(p, m, w);
@@ -1438,7 +1456,9 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
     uint32_t nseq = 0, nJ = 0, nt = 0, np = 0;
     bool ok = true, issued = false;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int m = item - (item / ipu) * ipu;
+      int u, m;
+      decode_item(p, item, u, m);
+      (void)u;
       for (int w = 0; ok && w < 2; ++w) {
         const int R0 = pair_seq_block(p, m, w);
         if (R0 < 0) break;
@@ -1536,7 +1556,8 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
     uint32_t np = 0, nseq = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int u = item / ipu, m = item - u * ipu;
+      int u, m;
+        decode_item(p, item, u, m);
       const Unit U = decode_unit(p, u);
       for (int w = 0; ok && w < 2; ++w) {
         const int R0 = pair_seq_block(p, m, w);
@@ -1624,7 +1645,8 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
     uint32_t nt = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      const int u = item / ipu, m = item - u * ipu;
+      int u, m;
+        decode_item(p, item, u, m);
       const Unit U = decode_unit(p, u);
       for (int w = 0; ok && w < 2; ++w) {
         const int R0 = pair_seq_block(p, m, w);
@@ -1740,9 +1762,13 @@ cudaError_t tc_launch_fwd(const TcParams& p, int d, int grid, cudaStream_t strea
   return d == 64 ? launch_fwd<64>(p, grid, stream) : launch_fwd<128>(p, grid, stream);
 }
 
-cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t stream) {
-  if (d == 64) return launch_bwd<64>(p, grid, stream);
+// `max_grid`: the number of SMs; the grid is one CTA per SM or one per work
+// item of the kernel chosen, whichever is fewer.
+cudaError_t tc_launch_bwd(const TcParams& p, int d, int max_grid, cudaStream_t stream) {
+  int grid = p.n_items < max_grid ? p.n_items : max_grid;
+  if (d == 64) return grid ? launch_bwd<64>(p, grid, stream) : cudaSuccess;
   if (p.nblk <= kPairMinBlocks - 1) {
+    if (!grid) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(relkl_bwd_tc64_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Bwd64Smem::ALLOC);
@@ -1752,9 +1778,11 @@ cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t strea
   }
   // work items of the pair kernel: ceil(npb / 2) per unit, npb = ceil(nblk / 2)
   TcParams q = p;
-  const int units = p.n_items / p.n_pairs;
   q.n_pairs = ((p.nblk + 1) / 2 + 1) / 2;
-  q.n_items = units * q.n_pairs;
+  q.n_local = q.part < q.n_pairs ? (q.n_pairs - q.part + q.n_parts - 1) / q.n_parts : 0;
+  q.n_items = q.n_units * q.n_local;
+  if (q.n_items == 0) return cudaSuccess;
+  grid = q.n_items < max_grid ? q.n_items : max_grid;
   cudaError_t e = cudaFuncSetAttribute(relkl_bwd_pair_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        BwdPairSmem::ALLOC);

@@ -118,12 +118,22 @@ def _arr(vals, ctype=ctypes.c_void_p):
     return (ctype * len(vals))(*[v if v is not None else None for v in vals])
 
 
+def _part(part) -> Tuple[int, int]:
+    p, n = (0, 1) if part is None else (int(part[0]), int(part[1]))
+    if n < 1 or not 0 <= p < n:
+        raise ValueError("part must be (index, count) with 0 <= index < count")
+    return p, n
+
+
 def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bool = True,
                   scale: float = 0.0, *, out: Optional[Sequence[Tuple[torch.Tensor, torch.Tensor]]] = None,
                   ws: Optional[torch.Tensor] = None, stream=None,
-                  lengths: Optional[torch.Tensor] = None):
+                  lengths: Optional[torch.Tensor] = None, part=None):
     """Forward over 1..3 relations in one launch.  Returns [(kl, stats)] per relation.
-    ``lengths``: optional int32 [B] valid lengths (right padding), shared by the relations."""
+    ``lengths``: optional int32 [B] valid lengths (right padding), shared by the relations.
+    ``part``: (index, count) to compute only that part of every unit's rows
+    (relkl_fwd_qkv_part); outputs allocated here are then zero elsewhere."""
+    p_idx, n_parts = _part(part)
     n = len(pairs)
     if not 1 <= n <= 3:
         raise ValueError("1 to 3 relations per call")
@@ -144,15 +154,19 @@ def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bo
             _check_out(kl, (B, H, N), "kl", dev)
             _check_out(st, (B, H, N, 4), "stats", dev)
         else:
-            kl = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-            st = torch.empty((B, H, N, 4), dtype=torch.float32, device=dev)
+            alloc = torch.empty if n_parts == 1 else torch.zeros
+            kl = alloc((B, H, N), dtype=torch.float32, device=dev)
+            st = alloc((B, H, N, 4), dtype=torch.float32, device=dev)
         outs.append((kl, st))
     ws = workspace(dev) if ws is None else ws
+    args = (n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
+            _arr([_ptr(o[0]) for o in outs]), _arr([_ptr(o[1]) for o in outs]))
+    tail = (_ptr(ws), ws.numel(), _stream(dev, stream))
     with torch.cuda.device(dev):
-        code = _abi.lib().relkl_fwd_qkv(
-            n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
-            _arr([_ptr(o[0]) for o in outs]), _arr([_ptr(o[1]) for o in outs]),
-            _ptr(ws), ws.numel(), _stream(dev, stream))
+        if n_parts == 1:
+            code = _abi.lib().relkl_fwd_qkv(*args, *tail)
+        else:
+            code = _abi.lib().relkl_fwd_qkv_part(*args, p_idx, n_parts, *tail)
     check(code, "relkl_fwd_qkv")
     return outs
 
@@ -161,8 +175,11 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
                   dkl: Optional[Sequence[Optional[torch.Tensor]]] = None, causal: bool = True,
                   scale: float = 0.0, *, out: Optional[Sequence[torch.Tensor]] = None,
                   ws: Optional[torch.Tensor] = None, stream=None,
-                  lengths: Optional[torch.Tensor] = None) -> List[torch.Tensor]:
-    """Backward over 1..3 relations in one launch.  Returns dX_s per relation (float32)."""
+                  lengths: Optional[torch.Tensor] = None, part=None) -> List[torch.Tensor]:
+    """Backward over 1..3 relations in one launch.  Returns dX_s per relation (float32).
+    ``part``: (index, count) to return only that part's rows' contribution to
+    dX_s (relkl_bwd_qkv_part); ``stats`` must then hold every row."""
+    p_idx, n_parts = _part(part)
     n = len(pairs)
     if not 1 <= n <= 3 or len(stats) != n:
         raise ValueError("1 to 3 relations per call, with one stats tensor each")
@@ -186,11 +203,14 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
         dxs.append(dx)
     ws = workspace(dev) if ws is None else ws
     dkl_arr = None if dkl is None else _arr([_ptr(g) for g in dkl])
+    args = (n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
+            _arr([_ptr(s) for s in stats]), dkl_arr, _arr([_ptr(d) for d in dxs]))
+    tail = (_ptr(ws), ws.numel(), _stream(dev, stream))
     with torch.cuda.device(dev):
-        code = _abi.lib().relkl_bwd_qkv(
-            n, descs, _arr([_ptr(p[0]) for p in pairs]), _arr([_ptr(p[1]) for p in pairs]),
-            _arr([_ptr(s) for s in stats]), dkl_arr, _arr([_ptr(d) for d in dxs]),
-            _ptr(ws), ws.numel(), _stream(dev, stream))
+        if n_parts == 1:
+            code = _abi.lib().relkl_bwd_qkv(*args, *tail)
+        else:
+            code = _abi.lib().relkl_bwd_qkv_part(*args, p_idx, n_parts, *tail)
     check(code, "relkl_bwd_qkv")
     return dxs
 

@@ -9,11 +9,11 @@ weight-gradient all-reduces outside this path.
 """
 from __future__ import annotations
 
-from typing import Tuple
+from typing import Dict, Tuple
 
 import torch
 
-__all__ = ["replica_seed", "shard_units", "max_over_ranks", "sum_over_ranks"]
+__all__ = ["replica_seed", "shard_units", "shard_heads", "max_over_ranks", "sum_over_ranks"]
 
 
 def replica_seed(base_seed: int, rank: int) -> int:
@@ -28,6 +28,21 @@ def shard_units(n_units: int, world: int, rank: int) -> Tuple[int, int]:
     q, r = divmod(n_units, world)
     start = rank * q + min(rank, r)
     return start, start + q + (1 if rank < r else 0)
+
+
+def shard_heads(pairs: Dict[str, Tuple[torch.Tensor, torch.Tensor]], world: int, rank: int
+                ) -> Dict[str, Tuple[torch.Tensor, torch.Tensor, int]]:
+    """This rank's share of one problem: for each relation {rel: (x_t, x_s)} of
+    [B, H_rel, N, d] tensors, the head range shard_units(H_rel, world, rank) as
+    strided views (no copy) plus the first head's index.  Relations with no
+    head on this rank are left out.  Each view is a valid desc for the fused
+    calls (same B and strides, H = the range's length, base moved by h0 heads)."""
+    out = {}
+    for rel, (xt, xs) in pairs.items():
+        h0, h1 = shard_units(int(xt.shape[1]), world, rank)
+        if h1 > h0:
+            out[rel] = (xt[:, h0:h1], xs[:, h0:h1], h0)
+    return out
 
 
 def _reduce(value: float, op, device) -> float:

@@ -357,6 +357,12 @@ def main():
     ap.add_argument("--chain", action="store_true",
                     help="time the chain rule to the Q/K/V weights (RoPE backward, weight "
                          "gradient GEMMs) at the LLaMA2-7B layer shape, N = 32768")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "units", "rows"],
+                    help="how N ranks share work: 'replicas' (default) runs one replica of the "
+                         "workload per rank (weak scaling); 'units' splits one problem's heads "
+                         "over the ranks; 'rows' splits every unit's rows (context parallel: "
+                         "token shards all-gathered, statistics all-reduced, dX reduce-"
+                         "scattered), both strong scaling")
     args = ap.parse_args()
     w = workload.get_config(args.config)
 
@@ -386,28 +392,67 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    # inputs: this rank's replica (seed offset by rank), resident in HBM
-    wr = workload.Workload(**{**w.__dict__, "seed": replica_seed(w.seed, rank)})
+    # inputs, resident in HBM: this rank's replica (seed offset by rank), or its
+    # share of one problem (the same seed on every rank)
+    split = args.split if world > 1 else "replicas"
+    wr = workload.Workload(**{**w.__dict__, "seed": replica_seed(w.seed, rank)
+                              if split == "replicas" else w.seed})
     t_gen = time.perf_counter()
     x = workload.generate(wr)
     t_gen = time.perf_counter() - t_gen
-    host = {r: (x[r][0].pin_memory(), x[r][1].pin_memory()) for r in w.relations}
-    pairs = [(host[r][0].to(dev), host[r][1].to(dev)) for r in w.relations]
+    rels = list(w.relations)
+    if split == "units":
+        from attention_relation_kl_b200.replicas import shard_heads
+        # this rank's heads of every relation (head-range views), copied as shards
+        sh = shard_heads(x, world, rank)
+        rels = [r for r in w.relations if r in sh]
+        x = {r: (sh[r][0].contiguous(), sh[r][1].contiguous()) for r in rels}
+    elif split == "rows":
+        if w.N % world:
+            raise SystemExit(f"--split rows needs N divisible by the rank count ({w.N}, {world})")
+        n_loc = w.N // world
+        # this rank's contiguous token shard, token-major [n_local, B, H, d]
+        x = {r: tuple(t.permute(2, 0, 1, 3)[rank * n_loc:(rank + 1) * n_loc].contiguous()
+                      for t in x[r]) for r in rels}
+    host = {r: (x[r][0].pin_memory(), x[r][1].pin_memory()) for r in rels}
+    del x
+    pairs = [(host[r][0].to(dev), host[r][1].to(dev)) for r in rels]
     in_bytes = sum(a.numel() * a.element_size() * 2 for a, _ in pairs)
     ws = rk.workspace(dev)
     stream = torch.cuda.current_stream(dev)
     torch.cuda.reset_peak_memory_stats(dev)
     base_alloc = torch.cuda.memory_allocated(dev)
 
-    outs = rk.relkl_fwd_qkv(pairs, w.causal, ws=ws)
-    dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, ws=ws)
+    if split == "rows":
+        from attention_relation_kl_b200.context_parallel import cp_backward, cp_forward
+        state = {}
+
+        def fwd():
+            state["full"], state["kl"], state["stats"] = cp_forward(pairs, w.causal)
+            return state["kl"]
+
+        def bwd():
+            state["dx"] = cp_backward(state["full"], state["stats"], w.causal)
+            return state["dx"]
+    else:
+        outs = rk.relkl_fwd_qkv(pairs, w.causal, ws=ws)
+        dxs = rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, ws=ws)
+
+        def fwd():
+            rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
+            return [o[0] for o in outs]
+
+        def bwd():
+            rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
+            return dxs
+    kl_out, dx_out = fwd(), bwd()
     torch.cuda.synchronize()
-    out_dx_bytes = sum(d.numel() * 4 for d in dxs)
-    stats_bytes = sum(o[0].numel() * 4 + o[1].numel() * 4 for o in outs)
+    out_dx_bytes = sum(d.numel() * 4 for d in dx_out)
+    stats_bytes = sum(k.numel() * 4 * 5 for k in kl_out)   # kl + 4 statistics per row
 
     def step():
-        rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
-        rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
+        fwd()
+        bwd()
 
     def stop_if_device_error(when):
         # every rank takes this collective, so that all leave together on an error
@@ -433,9 +478,9 @@ def main():
     t_start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
-        rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
+        fwd()
         ev[i][1].record(stream)
-        rk.relkl_bwd_qkv(pairs, [o[1] for o in outs], None, w.causal, out=dxs, ws=ws)
+        bwd()
         ev[i][2].record(stream)
     t_end.record(stream)
     barrier()
@@ -449,9 +494,9 @@ def main():
 
     # end to end through the public API with host buffers
     e2e_ms = None
-    h2d = sum(host[r][0].numel() * host[r][0].element_size() * 2 for r in w.relations)
-    host_dx = [torch.empty(d.shape, dtype=torch.float32, pin_memory=True) for d in dxs]
-    host_kl = [torch.empty(o[0].shape, dtype=torch.float32, pin_memory=True) for o in outs]
+    h2d = sum(host[r][0].numel() * host[r][0].element_size() * 2 for r in rels)
+    host_dx = [torch.empty(d.shape, dtype=torch.float32, pin_memory=True) for d in dx_out]
+    host_kl = [torch.empty(k.shape, dtype=torch.float32, pin_memory=True) for k in kl_out]
     d2h = sum(h.numel() * 4 for h in host_dx) + sum(h.numel() * 4 for h in host_kl)
     if args.e2e_steps > 0:
         barrier()
@@ -459,12 +504,12 @@ def main():
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.e2e_steps):
-            for (gt, gs), r in zip(pairs, w.relations):
+            for (gt, gs), r in zip(pairs, rels):
                 gt.copy_(host[r][0], non_blocking=True)
                 gs.copy_(host[r][1], non_blocking=True)
-            o = rk.relkl_fwd_qkv(pairs, w.causal, out=outs, ws=ws)
-            dd = rk.relkl_bwd_qkv(pairs, [q[1] for q in o], None, w.causal, out=dxs, ws=ws)
-            for hk, (kl, _) in zip(host_kl, o):
+            kk = fwd()
+            dd = bwd()
+            for hk, kl in zip(host_kl, kk):
                 hk.copy_(kl, non_blocking=True)
             for hd, dv in zip(host_dx, dd):
                 hd.copy_(dv, non_blocking=True)
@@ -473,10 +518,15 @@ def main():
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
 
     fl_fwd, fl_bwd = flops(w)
-    total_fl = (fl_fwd + fl_bwd) * world
+    copies = world if split == "replicas" else 1     # problems the job solves per step
+    total_fl = (fl_fwd + fl_bwd) * copies
     ms_step = ms / args.steps
     value = total_fl / (ms_step * 1e-3) / 1e12
-    tokens = w.B * w.N * world / (ms_step * 1e-3)
+    tokens = w.B * w.N * copies / (ms_step * 1e-3)
+    if split != "replicas":       # this rank's share of the flops, for its own kernel rates
+        share = (sum(a.shape[0] * a.shape[1] for a, _ in pairs) / (w.B * sum(w.heads(r) for r in
+                 w.relations)) if split == "units" else 1.0 / world)
+        fl_fwd, fl_bwd = fl_fwd * share, fl_bwd * share
 
     peaks, peak_src = load_peaks()
     tensor_path = w.dtype == "bf16" and w.d in (64, 128)
@@ -496,15 +546,17 @@ def main():
         result = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "weak" if split == "replicas" else "strong",
+            "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
                        "relations": "".join(w.relations), "causal": w.causal,
-                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "parallelism": (f"{split}{world}" if world > 1 else "single"),
                        "l2": f"inputs {in_bytes / 1e9:.2f} GB > L2 126 MB (no flush)"},
             "tokens_per_s": tokens,
             # the metric's "% of dense BF16 tensor peak": against the 2.25 PFLOP/s spec figure
             "pct_bf16_peak": 100.0 * value / (B200_DENSE_BF16_TFLOPS * world),
+            "split": split,
             # the same step against the measured cuBLAS bf16 GEMM rate (a plain library GEMM
             # under the power cap: sustained figure, the clocks it ran at are listed below)
             "pct_of_measured_cublas": 100.0 * value / (peak_tf * world),

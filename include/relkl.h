@@ -132,6 +132,36 @@ relkl_status relkl_bwd_qkv(int32_t n_rel, const relkl_desc* descs,
                            float* const* dx_s, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* One part of the fused calls above, for splitting one problem's rows over
+ * several GPUs (row-sharded context parallelism: the pages give the method
+ * for one device; this split follows from rows of the relation being
+ * independent in the forward and additive in the backward).
+ *
+ * Every unit's rows are grouped into work items (pairs of 128-row blocks on
+ * the tensor-core path, 32-row blocks on the CUDA-core path); part `part` of
+ * `n_parts` (0 <= part < n_parts) takes items part, part + n_parts, ...
+ * of every unit, so the parts hold nearly equal causal work.
+ *   relkl_fwd_qkv_part writes kl and stats for the rows of its items only and
+ *     leaves every other row untouched: zero the outputs, run every part and
+ *     add (or all-reduce) them to obtain relkl_fwd_qkv's result.
+ *   relkl_bwd_qkv_part needs stats for every row its items read (in general
+ *     all rows: combine the parts' forward statistics first).  dx_s is
+ *     overwritten with the contributions of this part's rows of G to both
+ *     sides of dX_s = scale (G + G^T) X_s; the sum of dx_s over all parts is
+ *     relkl_bwd_qkv's result.
+ * Teacher and student must hold every row of every unit (gather them first).
+ * n_parts = 1 is relkl_fwd_qkv / relkl_bwd_qkv.  RELKL_ERR_INVALID for a bad
+ * part index.                                                               */
+relkl_status relkl_fwd_qkv_part(int32_t n_rel, const relkl_desc* descs,
+                                const void* const* x_t, const void* const* x_s,
+                                float* const* kl, float* const* stats, int32_t part,
+                                int32_t n_parts, void* ws, size_t ws_bytes, void* stream);
+relkl_status relkl_bwd_qkv_part(int32_t n_rel, const relkl_desc* descs,
+                                const void* const* x_t, const void* const* x_s,
+                                const float* const* stats, const float* const* dkl,
+                                float* const* dx_s, int32_t part, int32_t n_parts, void* ws,
+                                size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then reads the workspace record.  Returns RELKL_OK
  * or RELKL_ERR_TIMEOUT; *where (if not NULL) receives the code of the wait
  * that ran out (0 when none).                                                */

@@ -46,7 +46,7 @@ import numpy as np
 import torch
 
 __all__ = ["as_f64", "relation_logits", "allowed", "fwd_unit", "bwd_unit",
-           "fwd_rows", "bwd_rows", "fwd", "bwd", "unit_loss", "relation_probs"]
+           "fwd_rows", "bwd_rows", "fwd", "bwd", "unit_loss", "relation_probs", "bwd_contrib"]
 
 
 def as_f64(x) -> np.ndarray:
@@ -243,3 +243,31 @@ def relation_probs(xt, xs, causal: bool = True, scale: Optional[float] = None):
     logp_t, _, _ = _masked_log_softmax(relation_logits(xt, xt, s), ok)
     logp_s, _, _ = _masked_log_softmax(relation_logits(xs, xs, s), ok)
     return np.where(ok, np.exp(logp_t), 0.0), np.where(ok, np.exp(logp_s), 0.0)
+
+
+def bwd_contrib(xt, xs, rows: Iterable[int], dkl=None, causal: bool = True,
+                scale: Optional[float] = None) -> np.ndarray:
+    """The share of dL/dX_s that the given rows of G produce.
+
+    dX_s = s (G + G^T) X_s is linear in G, and G's rows are formed
+    independently (row i needs only row i's logits and LSEs), so dX_s is the
+    sum over rows i of s (e_i G(i,:) X_s + G(i,:)^T X_s[i]): the first term
+    lands on row i, the second on every column row j that row i sees.  This
+    returns that sum over ``rows`` only; summing it over a partition of the
+    rows gives ``bwd_unit``.
+    """
+    xt, xs = as_f64(xt), as_f64(xs)
+    rows = np.asarray(list(rows), dtype=np.int64)
+    N, d = xt.shape
+    s = _scale(d, scale)
+    g_up = _default_dkl(dkl, N)
+    dx = np.zeros_like(xs)
+    if rows.size == 0:
+        return dx
+    ok = allowed(rows, N, causal)
+    logp_t, _, _ = _masked_log_softmax(relation_logits(xt[rows], xt, s), ok)
+    logp_s, _, _ = _masked_log_softmax(relation_logits(xs[rows], xs, s), ok)
+    g = g_up[rows, None] * np.where(ok, np.exp(logp_s) - np.exp(logp_t), 0.0)
+    dx[rows] += s * (g @ xs)              # row side
+    dx += s * (g.T @ xs[rows])            # column side
+    return dx

@@ -385,3 +385,28 @@ def test_lengths_match_torch_key_padding_mask(causal):
     np.testing.assert_allclose(r["kl"], kl_ref.numpy(), rtol=1e-10, atol=1e-13)
     np.testing.assert_allclose(dense.bwd(xt, xs, None, causal, lengths=np.array(lengths)),
                                xs_var.grad.numpy(), rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_row_partition_contributions_sum_to_the_gradient(causal):
+    """dX_s is linear in G and G's rows are independent: the contributions of
+    the rows of any partition add up to the whole gradient (the basis of
+    splitting one unit's rows over devices), and one part alone is not it."""
+    N, d = 23, 8
+    xt, xs = _rand_pair(N, d, seed=91)
+    dkl = np.linspace(-0.5, 1.0, N)
+    full = dense.bwd_unit(xt, xs, dkl, causal)
+    rng = np.random.default_rng(4)
+    owner = rng.integers(0, 3, size=N)
+    parts = [dense.bwd_contrib(xt, xs, np.flatnonzero(owner == k), dkl, causal) for k in range(3)]
+    np.testing.assert_allclose(sum(parts), full, rtol=1e-12, atol=1e-15)
+    assert np.abs(parts[0] - full).max() > 1e-3 * np.abs(full).max()
+    # one part's rows: its row side and column side, written out for one row
+    i = int(np.flatnonzero(owner == 1)[0])
+    one = dense.bwd_contrib(xt, xs, [i], dkl, causal)
+    s = 1.0 / math.sqrt(d)
+    p_t, p_s = dense.relation_probs(xt, xs, causal)
+    g_i = dkl[i] * (p_s[i] - p_t[i])
+    want = np.outer(g_i, xs[i]) * s
+    want[i] += s * (g_i @ xs)
+    np.testing.assert_allclose(one, want, rtol=1e-12, atol=1e-15)
