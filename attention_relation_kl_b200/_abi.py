@@ -28,7 +28,9 @@ class relkl_desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("stride", ctypes.c_int64 * 4), ("dtype", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("scale", ctypes.c_float),
-                ("reserved", ctypes.c_int32), ("lengths", ctypes.c_void_p)]
+                ("reserved", ctypes.c_int32), ("lengths", ctypes.c_void_p),
+                ("cu_seqlens", ctypes.c_void_p), ("n_seq", ctypes.c_int32),
+                ("max_seqlen", ctypes.c_int32)]
 
 
 class relkl_rope(ctypes.Structure):

@@ -103,7 +103,11 @@ relkl_status device_info(DevInfo* out) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int64_t n_units(const relkl_desc& d) { return static_cast<int64_t>(d.B) * d.H; }
+// Units of a desc: (b, h) of its [B, H, N, d] tensors, or (sequence, head)
+// of packed sequences.
+int64_t n_units(const relkl_desc& d) {
+  return static_cast<int64_t>(d.cu_seqlens ? d.n_seq : d.B) * d.H;
+}
 
 relkl_status check_desc(const relkl_desc* d) {
   if (!d) return RELKL_ERR_INVALID;
@@ -112,13 +116,20 @@ relkl_status check_desc(const relkl_desc* d) {
   if (d->causal != 0 && d->causal != 1) return RELKL_ERR_INVALID;
   if (d->reserved != 0) return RELKL_ERR_INVALID;
   if (d->lengths && !aligned(d->lengths, 4)) return RELKL_ERR_INVALID;
+  if (d->cu_seqlens) {
+    if (!aligned(d->cu_seqlens, 4) || d->lengths || d->B != 1 || d->n_seq < 0 ||
+        d->max_seqlen < 0 || d->max_seqlen > d->N)
+      return RELKL_ERR_INVALID;
+  } else if (d->n_seq != 0 || d->max_seqlen != 0) {
+    return RELKL_ERR_INVALID;
+  }
   if (!(d->scale >= 0.f) || !std::isfinite(d->scale)) return RELKL_ERR_INVALID;
   if (d->stride[3] != 1) return RELKL_ERR_INVALID;
   for (int i = 0; i < 3; ++i)
     if (d->stride[i] < 0) return RELKL_ERR_INVALID;
   if (d->d > 128) return RELKL_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->N) * d->d >= (int64_t(1) << 31)) return RELKL_ERR_UNSUPPORTED;
-  if (n_units(*d) * d->N >= (int64_t(1) << 40)) return RELKL_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->B) * d->H * d->N >= (int64_t(1) << 40)) return RELKL_ERR_UNSUPPORTED;
   return RELKL_OK;
 }
 
@@ -192,12 +203,13 @@ relkl_status check_multi(int32_t n_rel, const relkl_desc* descs, const void* con
     const relkl_desc& a = descs[0];
     const relkl_desc& b = descs[r];
     if (a.N != b.N || a.d != b.d || a.dtype != b.dtype || a.causal != b.causal ||
-        a.scale != b.scale)
+        a.scale != b.scale || (a.cu_seqlens == nullptr) != (b.cu_seqlens == nullptr) ||
+        a.max_seqlen != b.max_seqlen)
       return RELKL_ERR_INVALID;
     units += n_units(b);
   }
   if (units >= (int64_t(1) << 30)) return RELKL_ERR_UNSUPPORTED;
-  *empty = (units == 0 || descs[0].N == 0);
+  *empty = (units == 0 || descs[0].N == 0 || (descs[0].cu_seqlens && descs[0].max_seqlen == 0));
   if (*empty) return RELKL_OK;
   for (int r = 0; r < n_rel; ++r) {
     if (n_units(descs[r]) == 0) continue;
@@ -227,16 +239,20 @@ relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const*
     relkl_status st = encode_x(&s.tm_t, descs[r], xt[r]);
     if (st != RELKL_OK) return st;
     if ((st = encode_x(&s.tm_s, descs[r], xs[r])) != RELKL_OK) return st;
-    s.B = descs[r].B;
+    s.B = descs[r].cu_seqlens ? descs[r].n_seq : descs[r].B;
     s.H = descs[r].H;
     s.lengths = descs[r].lengths;
+    s.cu_seqlens = descs[r].cu_seqlens;
+    s.max_seqlen = descs[r].max_seqlen;
     s.unit_begin = ub;
     ub += static_cast<int>(n_units(descs[r]));
     ++seg;
   }
   p->n_seg = seg;
   p->N = d0.N;
-  p->nblk = (d0.N + 127) / 128;
+  // rows a unit's work covers: every row, or at most max_seqlen of a packed sequence
+  const int span = d0.cu_seqlens ? d0.max_seqlen : d0.N;
+  p->nblk = (span + 127) / 128;
   p->n_pairs = (p->nblk + 1) / 2;
   p->n_units = ub;
   p->part = part;
@@ -264,9 +280,11 @@ relkl_status build_simt(int32_t n_rel, const relkl_desc* descs, const void* cons
     s.sb = descs[r].stride[0];
     s.sh = descs[r].stride[1];
     s.sn = descs[r].stride[2];
-    s.B = descs[r].B;
+    s.B = descs[r].cu_seqlens ? descs[r].n_seq : descs[r].B;
     s.H = descs[r].H;
     s.lengths = descs[r].lengths;
+    s.cu_seqlens = descs[r].cu_seqlens;
+    s.max_seqlen = descs[r].max_seqlen;
     s.unit_begin = ub;
     ub += static_cast<int>(n_units(descs[r]));
     ++seg;
@@ -280,7 +298,7 @@ relkl_status build_simt(int32_t n_rel, const relkl_desc* descs, const void* cons
   p->n_units = ub;
   p->part = part;
   p->n_parts = n_parts;
-  const int nblk32 = (d0.N + 31) / 32;
+  const int nblk32 = ((d0.cu_seqlens ? d0.max_seqlen : d0.N) + 31) / 32;
   p->nblk_local = part < nblk32 ? (nblk32 - part + n_parts - 1) / n_parts : 0;
   return RELKL_OK;
 }
@@ -399,7 +417,8 @@ relkl_status bwd_impl(int32_t n_rel, const relkl_desc* descs, const void* const*
   // dX_s is accumulated with atomics: clear it first (same stream)
   for (int r = 0; r < n_rel; ++r) {
     if (!n_units(descs[r])) continue;
-    const int64_t n = n_units(descs[r]) * descs[r].N * descs[r].d;
+    // the whole [B, H, N, d] tensor (packed sequences: B = 1, every token)
+    const int64_t n = static_cast<int64_t>(descs[r].B) * descs[r].H * descs[r].N * descs[r].d;
     if ((e = launch_zero(dx_s[r], n, dev.sms, st)) != cudaSuccess) return cuda_fail(e);
   }
   if (tc) {

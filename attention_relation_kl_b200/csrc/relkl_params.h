@@ -23,9 +23,10 @@ struct TcSeg {
   const float* dkl;          // [B,H,N] or null (1/N)
   float* dx;                 // [B,H,N,d] float32
   const int* lengths;        // [B] valid lengths (device) or null (all N)
-  int B, H;
+  const int* cu_seqlens;     // packed sequences: [n_seq + 1] token offsets (device), or null
+  int B, H;                  // packed sequences: B = n_seq (units are (sequence, head))
   int unit_begin;
-  int pad_;
+  int max_seqlen;            // packed sequences: bound on every sequence's length
 };
 
 struct TcParams {
@@ -57,9 +58,10 @@ struct SimtSeg {
   const float* dkl;
   float* dx;
   const int* lengths;        // [B] valid lengths (device) or null (all N)
-  int B, H;
+  const int* cu_seqlens;     // packed sequences: [n_seq + 1] token offsets, or null
+  int B, H;                  // packed sequences: B = n_seq
   int unit_begin;
-  int pad_;
+  int max_seqlen;
 };
 
 struct SimtParams {

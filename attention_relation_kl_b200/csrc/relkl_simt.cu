@@ -24,11 +24,14 @@ __device__ __forceinline__ float load_x(const void* base, int is_bf16, int64_t o
 
 struct SimtUnit {
   const SimtSeg* seg;
-  int64_t xoff;   // element offset of the unit's [N, d] slice in x
+  int64_t xoff;   // element offset of the unit's first row in x
   int64_t row0;   // first row of the unit in [B,H,N] arrays
   int L;          // valid rows and columns (its batch element's length, or N)
+  int span;       // rows the unit covers: its length for a packed sequence, else N
 };
 
+// Unit u: (b, h) of a batched relation, or (sequence k, head h) of packed
+// sequences (sequence k on tokens [cu_seqlens[k], cu_seqlens[k+1]) of [1,H,N,d]).
 __device__ __forceinline__ SimtUnit simt_unit(const SimtParams& p, int u) {
   int r = 0;
   for (int k = 1; k < p.n_seg; ++k)
@@ -38,9 +41,19 @@ __device__ __forceinline__ SimtUnit simt_unit(const SimtParams& p, int u) {
   const int b = local / s->H, h = local - (local / s->H) * s->H;
   SimtUnit out;
   out.seg = s;
-  out.xoff = b * s->sb + h * s->sh;
-  out.row0 = (static_cast<int64_t>(b) * s->H + h) * p.N;
-  out.L = s->lengths ? max(0, min(p.N, s->lengths[b])) : p.N;   // valid rows and columns
+  if (s->cu_seqlens) {
+    const int a = min(max(s->cu_seqlens[b], 0), p.N);
+    const int e = min(max(s->cu_seqlens[b + 1], a), p.N);
+    out.L = min(e - a, s->max_seqlen);
+    out.span = out.L;
+    out.xoff = h * s->sh + a * s->sn;
+    out.row0 = static_cast<int64_t>(h) * p.N + a;
+  } else {
+    out.L = s->lengths ? max(0, min(p.N, s->lengths[b])) : p.N;   // valid rows and columns
+    out.span = p.N;
+    out.xoff = b * s->sb + h * s->sh;
+    out.row0 = (static_cast<int64_t>(b) * s->H + h) * p.N;
+  }
   return out;
 }
 
@@ -64,7 +77,6 @@ relkl_fwd_simt_kernel(const __grid_constant__ SimtParams p) {
   float* xtj = xsi + SB * pitch;
   float* xsj = xtj + SB * pitch;
 
-  const int nblk = (p.N + SB - 1) / SB;
   // this call's 32-row blocks of the unit: part, part + n_parts, ...
   const int u = blockIdx.x / p.nblk_local;
   const int I = p.part + (blockIdx.x - u * p.nblk_local) * p.n_parts;
@@ -74,15 +86,16 @@ relkl_fwd_simt_kernel(const __grid_constant__ SimtParams p) {
   const int row = I * SB + rr;
   const float sc = p.scale;
 
-  stage_rows(xti, S.xt, p.is_bf16, U.xoff, S.sn, I * SB, p.N, d);
-  stage_rows(xsi, S.xs, p.is_bf16, U.xoff, S.sn, I * SB, p.N, d);
+  if (I * SB >= U.span) return;   // a block past a short packed sequence
+  stage_rows(xti, S.xt, p.is_bf16, U.xoff, S.sn, I * SB, U.span, d);
+  stage_rows(xsi, S.xs, p.is_bf16, U.xoff, S.sn, I * SB, U.span, d);
 
   float m_run = -INFINITY, St = 0.f, C = 0.f, A = 0.f;
-  const int nJ = p.causal ? I + 1 : nblk;
+  const int nJ = p.causal ? I + 1 : (U.span + SB - 1) / SB;
   for (int J = 0; J < nJ; ++J) {
     __syncthreads();
-    stage_rows(xtj, S.xt, p.is_bf16, U.xoff, S.sn, J * SB, p.N, d);
-    stage_rows(xsj, S.xs, p.is_bf16, U.xoff, S.sn, J * SB, p.N, d);
+    stage_rows(xtj, S.xt, p.is_bf16, U.xoff, S.sn, J * SB, U.span, d);
+    stage_rows(xsj, S.xs, p.is_bf16, U.xoff, S.sn, J * SB, U.span, d);
     __syncthreads();
     float zt[4], zs[4];
     bool ok[4];
@@ -125,10 +138,10 @@ relkl_fwd_simt_kernel(const __grid_constant__ SimtParams p) {
     C += __shfl_xor_sync(0xffffffffu, C, o);
     A += __shfl_xor_sync(0xffffffffu, A, o);
   }
-  if (cg == 0 && row < p.N && row >= U.L) {   // padding row
+  if (cg == 0 && row < U.span && row >= U.L) {   // padding row
     S.kl[U.row0 + row] = 0.f;
     reinterpret_cast<float4*>(S.stats)[U.row0 + row] = make_float4(0.f, 0.f, 0.f, 0.f);
-  } else if (cg == 0 && row < p.N) {
+  } else if (cg == 0 && row < U.span) {
     const float lse_t = m_run + logf(St);
     const float l1 = log1pf(C / St);
     const float w = A / St;
@@ -148,7 +161,6 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
   float* xsj = xtj + SB * pitch;
   float* g = xsj + SB * pitch;      // [32][33]
 
-  const int nblk = (p.N + SB - 1) / SB;
   // this call's 32-row blocks of the unit: part, part + n_parts, ...
   const int u = blockIdx.x / p.nblk_local;
   const int I = p.part + (blockIdx.x - u * p.nblk_local) * p.n_parts;
@@ -158,8 +170,9 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
   const int row = I * SB + rr;
   const float sc = p.scale;
 
-  stage_rows(xti, S.xt, p.is_bf16, U.xoff, S.sn, I * SB, p.N, d);
-  stage_rows(xsi, S.xs, p.is_bf16, U.xoff, S.sn, I * SB, p.N, d);
+  if (I * SB >= U.span) return;   // a block past a short packed sequence
+  stage_rows(xti, S.xt, p.is_bf16, U.xoff, S.sn, I * SB, U.span, d);
+  stage_rows(xsi, S.xs, p.is_bf16, U.xoff, S.sn, I * SB, U.span, d);
   float lse_t = 0.f, lse_s = 0.f, mul = 0.f;
   if (row < U.L) {
     const float4 st4 = reinterpret_cast<const float4*>(S.stats)[U.row0 + row];
@@ -173,11 +186,11 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
 #pragma unroll
   for (int m = 0; m < MAXC; ++m) acc[m] = 0.f;
 
-  const int nJ = p.causal ? I + 1 : nblk;
+  const int nJ = p.causal ? I + 1 : (U.span + SB - 1) / SB;
   for (int J = 0; J < nJ; ++J) {
     __syncthreads();
-    stage_rows(xtj, S.xt, p.is_bf16, U.xoff, S.sn, J * SB, p.N, d);
-    stage_rows(xsj, S.xs, p.is_bf16, U.xoff, S.sn, J * SB, p.N, d);
+    stage_rows(xtj, S.xt, p.is_bf16, U.xoff, S.sn, J * SB, U.span, d);
+    stage_rows(xsj, S.xs, p.is_bf16, U.xoff, S.sn, J * SB, U.span, d);
     __syncthreads();
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -203,7 +216,7 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
     }
     // dX[J] += G^T X_s[I]   (thread: column-block row jj = rr)
     const int jrow = J * SB + rr;
-    if (jrow < p.N) {
+    if (jrow < U.span) {
       float* dst = S.dx + (U.row0 + jrow) * d;
       for (int k = cg; k < d; k += 8) {
         float a = 0.f;
@@ -212,7 +225,7 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
       }
     }
   }
-  if (row < p.N) {
+  if (row < U.span) {
     float* dst = S.dx + (U.row0 + row) * d;
 #pragma unroll
     for (int m = 0; m < MAXC; ++m) {

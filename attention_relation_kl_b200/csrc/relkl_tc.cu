@@ -53,10 +53,19 @@ constexpr unsigned long long kDrainNs = 200000000ull;  // 0.2 s for in-flight co
 
 struct Unit {
   const TcSeg* seg;
-  int b, h;
-  long long row0;  // (b*H + h) * N : first row of the unit in [B,H,N] arrays
+  int b, h;        // TMA batch and head coordinates
+  long long row0;  // first row of the unit in the [B,H,N] arrays (kl, stats, dkl)
+  int tok0;        // TMA row coordinate of the unit's first row (packed sequences), else 0
+  int len;         // valid rows and columns of the unit
+  int span;        // rows the unit's work items cover: len for packed sequences, else N
+  int nblk;        // ceil(span / 128)
 };
 
+// Unit u of the launch.  Units of a batched relation are (b, h) of its
+// [B, H, N, d] tensors, right-padded to a per-batch length when lengths are
+// given; units of packed sequences are (sequence k, head h) of [1, H, N, d]
+// tensors holding the sequences back to back, sequence k on tokens
+// [cu_seqlens[k], cu_seqlens[k+1]).
 __device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
   int r = 0;
 #pragma unroll
@@ -66,9 +75,25 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
   const int local = u - s->unit_begin;
   Unit out;
   out.seg = s;
-  out.b = local / s->H;
-  out.h = local - out.b * s->H;
-  out.row0 = (static_cast<long long>(out.b) * s->H + out.h) * p.N;
+  if (s->cu_seqlens) {
+    const int k = local / s->H;
+    out.b = 0;
+    out.h = local - k * s->H;
+    const int a = min(max(s->cu_seqlens[k], 0), p.N);
+    const int e = min(max(s->cu_seqlens[k + 1], a), p.N);
+    out.tok0 = a;
+    out.len = min(e - a, s->max_seqlen);
+    out.span = out.len;
+    out.row0 = static_cast<long long>(out.h) * p.N + a;
+  } else {
+    out.b = local / s->H;
+    out.h = local - out.b * s->H;
+    out.tok0 = 0;
+    out.len = s->lengths ? max(0, min(p.N, s->lengths[out.b])) : p.N;
+    out.span = p.N;
+    out.row0 = (static_cast<long long>(out.b) * s->H + out.h) * p.N;
+  }
+  out.nblk = (out.span + BM - 1) / BM;
   return out;
 }
 
@@ -80,20 +105,17 @@ __device__ __forceinline__ void decode_item(const TcParams& p, int item, int& u,
 }
 
 // Row blocks of one work item: pass 0 is the longer block nblk-1-p, pass 1
-// (absent when both coincide) is block p.
-// Valid rows and columns of unit U: its batch element's length, or all N.
-__device__ __forceinline__ int unit_len(const TcParams& p, const Unit& U) {
-  const int* len = U.seg->lengths;
-  return len ? max(0, min(p.N, len[U.b])) : p.N;
+// (absent when both coincide) is block p.  An item index past the unit's
+// own pair count (a short packed sequence) has no pass.
+__device__ __forceinline__ int item_passes(const Unit& U, int pp) {
+  if (pp >= (U.nblk + 1) / 2) return 0;
+  return (pp == U.nblk - 1 - pp) ? 1 : 2;
 }
-__device__ __forceinline__ int item_passes(const TcParams& p, int pp) {
-  return (pp == p.nblk - 1 - pp) ? 1 : 2;
+__device__ __forceinline__ int pass_block(const Unit& U, int pp, int pass) {
+  return pass == 0 ? U.nblk - 1 - pp : pp;
 }
-__device__ __forceinline__ int pass_block(const TcParams& p, int pp, int pass) {
-  return pass == 0 ? p.nblk - 1 - pp : pp;
-}
-__device__ __forceinline__ int n_col_tiles(const TcParams& p, int I) {
-  return p.causal ? I + 1 : p.nblk;
+__device__ __forceinline__ int n_col_tiles(const TcParams& p, const Unit& U, int I) {
+  return p.causal ? I + 1 : U.nblk;
 }
 
 // Issue the K-loop of one M=128 x N=128 logit tile: acc = A_tile * B_tile^T
@@ -210,17 +232,17 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
         int u, pp;
         decode_item(p, item, u, pp);
         const Unit U = decode_unit(p, u);
-        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-          const int I = pass_block(p, pp, pass);
+        for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+          const int I = pass_block(U, pp, pass);
           if (!(ok = mbar_wait(EMPTY_I, (nI & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
           mbar_arrive_expect_tx(FULL_I, 2 * L::TILE);
 #pragma unroll
           for (int b = 0; b < D / 64; ++b) {
-            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, I * BM, U.h, U.b);
-            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, I * BM, U.h, U.b);
+            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, U.tok0 + I * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, U.tok0 + I * BM, U.h, U.b);
           }
           ++nI;
-          const int nT = n_col_tiles(p, I);
+          const int nT = n_col_tiles(p, U, I);
           for (int J = 0; J < nT; ++J) {
             const int st = nJ & 1;
             if (!(ok = mbar_wait(EMPTY_J(st), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
@@ -228,9 +250,9 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
             mbar_arrive_expect_tx(FULL_J(st), 2 * L::TILE);
 #pragma unroll
             for (int b = 0; b < D / 64; ++b) {
-              tma_load_4d(xt + b * BOX, &U.seg->tm_t, FULL_J(st), b * 64, J * BN, U.h, U.b);
-              tma_load_4d(xt + L::TILE + b * BOX, &U.seg->tm_s, FULL_J(st), b * 64, J * BN, U.h,
-                          U.b);
+              tma_load_4d(xt + b * BOX, &U.seg->tm_t, FULL_J(st), b * 64, U.tok0 + J * BN, U.h, U.b);
+              tma_load_4d(xt + L::TILE + b * BOX, &U.seg->tm_s, FULL_J(st), b * 64, U.tok0 + J * BN,
+                          U.h, U.b);
             }
             ++nJ;
           }
@@ -258,11 +280,11 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         int u, pp;
         decode_item(p, item, u, pp);
-        (void)u;
-        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-          const int I = pass_block(p, pp, pass);
+        const Unit U = decode_unit(p, u);
+        for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+          const int I = pass_block(U, pp, pass);
           if (!(ok = mbar_wait_warp(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
-          const int nT = n_col_tiles(p, I);
+          const int nT = n_col_tiles(p, U, I);
           for (int J = 0; J < nT; ++J) {
             const int st = nJ & 1;
             const int buf = nt & 1;
@@ -302,11 +324,11 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
       int u, pp;
         decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
-      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-        const int I = pass_block(p, pp, pass);
+      for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+        const int I = pass_block(U, pp, pass);
         const int row = I * BM + r;
-        const int nT = n_col_tiles(p, I);
-        const int L = unit_len(p, U);
+        const int nT = n_col_tiles(p, U, I);
+        const int L = U.len;
         float m_run = -INFINITY;
         // running sums, two float2 lanes each: S_t, C = sum(e_s - e_t), A = sum e_t (z_t - z_s)
         float2 S2[2], C2[2], A2[2];
@@ -440,7 +462,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
             const float w = p.scale * At / St;
             U.seg->kl[g] = w + l1;
             reinterpret_cast<float4*>(U.seg->stats)[g] = make_float4(mz, lse_t, lse_t + l1, w);
-          } else if (row < p.N) {   // padding row
+          } else if (row < U.span) {   // padding row (a packed sequence has none: span = len)
             U.seg->kl[g] = 0.f;
             reinterpret_cast<float4*>(U.seg->stats)[g] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
@@ -595,17 +617,17 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
         int u, pp;
         decode_item(p, item, u, pp);
         const Unit U = decode_unit(p, u);
-        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-          const int I = pass_block(p, pp, pass);
+        for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+          const int I = pass_block(U, pp, pass);
           if (!(ok = mbar_wait(EMPTY_I, (nI & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
           mbar_arrive_expect_tx(FULL_I, 2 * L::TILE);
 #pragma unroll
           for (int b = 0; b < D / 64; ++b) {
-            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, I * BM, U.h, U.b);
-            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, I * BM, U.h, U.b);
+            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, U.tok0 + I * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, U.tok0 + I * BM, U.h, U.b);
           }
           ++nI;
-          const int nT = n_col_tiles(p, I);
+          const int nT = n_col_tiles(p, U, I);
           for (int J = 0; J < nT; ++J) {
             // teacher tile first: its single slot frees as soon as Z_t(J-1) is done,
             // while a student slot frees only after the gradient MMAs of J-2
@@ -613,8 +635,8 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
             mbar_arrive_expect_tx(FULL_T, L::TILE);
 #pragma unroll
             for (int b = 0; b < D / 64; ++b)
-              tma_load_4d(base + L::XT_R + b * BOX, &U.seg->tm_t, FULL_T, b * 64, J * BN, U.h,
-                          U.b);
+              tma_load_4d(base + L::XT_R + b * BOX, &U.seg->tm_t, FULL_T, b * 64, U.tok0 + J * BN,
+                          U.h, U.b);
             ++armsT;
             const int st = nJ & 1;
             if (!(ok = mbar_wait(EMPTY_S(st), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
@@ -622,7 +644,7 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
             for (int b = 0; b < D / 64; ++b)
               tma_load_4d(base + L::XS_R + st * L::TILE + b * BOX, &U.seg->tm_s, FULL_S(st),
-                          b * 64, J * BN, U.h, U.b);
+                          b * 64, U.tok0 + J * BN, U.h, U.b);
             ++armsS[st];
             ++nJ;
           }
@@ -674,11 +696,11 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         int u, pp;
         decode_item(p, item, u, pp);
-        (void)u;
-        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-          const int I = pass_block(p, pp, pass);
+        const Unit U = decode_unit(p, u);
+        for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+          const int I = pass_block(U, pp, pass);
           if (!(ok = mbar_wait(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
-          const int nT = n_col_tiles(p, I);
+          const int nT = n_col_tiles(p, U, I);
           int prev_st = -1;
           for (int J = 0; J < nT; ++J) {
             const int st = nJ & 1;
@@ -722,15 +744,15 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       int u, pp;
         decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
-      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-        const int I = pass_block(p, pp, pass);
-        const int nT = n_col_tiles(p, I);
+      for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+        const int I = pass_block(U, pp, pass);
+        const int nT = n_col_tiles(p, U, I);
         for (int J = 0; J < nT; ++J) {
           ok = mbar_wait(P_FULL, np & 1, wc, W_EPI_P_FULL);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
-          epilogue_reduce<D>(tmem + lane_addr + T_P, stg, nstg, &U.seg->tm_dx, J * BN + q * 32,
+          epilogue_reduce<D>(tmem + lane_addr + T_P, stg, nstg, &U.seg->tm_dx, U.tok0 + J * BN + q * 32,
                              U.h, U.b, p.N, lane, P_EMPTY);
           ++np;
         }
@@ -739,7 +761,7 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        epilogue_reduce<D>(tmem + lane_addr + T_DXI, stg, nstg, &U.seg->tm_dx, I * BM + q * 32,
+        epilogue_reduce<D>(tmem + lane_addr + T_DXI, stg, nstg, &U.seg->tm_dx, U.tok0 + I * BM + q * 32,
                            U.h, U.b, p.N, lane, DXI_EMPTY);
         ++nrb;
       }
@@ -760,10 +782,10 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
       int u, pp;
         decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
-      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-        const int I = pass_block(p, pp, pass);
+      for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+        const int I = pass_block(U, pp, pass);
         const int row = I * BM + r;
-        const int L = unit_len(p, U);
+        const int L = U.len;
         const bool rvalid = row < L;
         float bt = 0.f, bs = 0.f, mul = 0.f;
         if (rvalid) {
@@ -774,7 +796,7 @@ relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
           mul = up * p.scale;   // the logit scale of dX_s is folded into G
         }
         const int lim = !rvalid ? -1 : (p.causal ? min(row, L - 1) : L - 1);
-        const int nT = n_col_tiles(p, I);
+        const int nT = n_col_tiles(p, U, I);
         for (int J = 0; J < nT; ++J) {
           ok = mbar_wait(S_FULL, ns & 1, wc, W_SM_S_FULL);
           ok = __all_sync(0xffffffffu, ok);
@@ -870,8 +892,8 @@ static_assert(Bwd64Smem::ALLOC <= 232448, "backward shared memory exceeds 227 KB
 
 constexpr int BN64 = 64;
 
-__device__ __forceinline__ int n_col_tiles64(const TcParams& p, int I) {
-  const int nb64 = (p.N + BN64 - 1) / BN64;
+__device__ __forceinline__ int n_col_tiles64(const TcParams& p, const Unit& U, int I) {
+  const int nb64 = (U.span + BN64 - 1) / BN64;
   return p.causal ? min(2 * I + 2, nb64) : nb64;
 }
 
@@ -954,17 +976,17 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
         int u, pp;
         decode_item(p, item, u, pp);
         const Unit U = decode_unit(p, u);
-        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-          const int I = pass_block(p, pp, pass);
+        for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+          const int I = pass_block(U, pp, pass);
           if (!(ok = mbar_wait(EMPTY_I, (nI & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
           mbar_arrive_expect_tx(FULL_I, 2 * L::TILE_I);
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
-            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, I * BM, U.h, U.b);
-            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, I * BM, U.h, U.b);
+            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, U.tok0 + I * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, U.tok0 + I * BM, U.h, U.b);
           }
           ++nI;
-          const int nT = n_col_tiles64(p, I);
+          const int nT = n_col_tiles64(p, U, I);
           for (int J = 0; J < nT; ++J) {
             const int tt = nJ & 1, ts = nJ & 3;
             if (!(ok = mbar_wait(EMPTY_T(tt), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
@@ -972,14 +994,14 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
             for (int b = 0; b < 2; ++b)
               tma_load_4d(base + L::XT_R + tt * L::TILE_J + b * L::BOX_J, &U.seg->tm_t64,
-                          FULL_T(tt), b * 64, J * BN64, U.h, U.b);
+                          FULL_T(tt), b * 64, U.tok0 + J * BN64, U.h, U.b);
             ++armsT[tt];
             if (!(ok = mbar_wait(EMPTY_S(ts), ((nJ >> 2) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
             mbar_arrive_expect_tx(FULL_S(ts), L::TILE_J);
 #pragma unroll
             for (int b = 0; b < 2; ++b)
               tma_load_4d(base + L::XS_R + ts * L::TILE_J + b * L::BOX_J, &U.seg->tm_s64,
-                          FULL_S(ts), b * 64, J * BN64, U.h, U.b);
+                          FULL_S(ts), b * 64, U.tok0 + J * BN64, U.h, U.b);
             ++armsS[ts];
             ++nJ;
           }
@@ -1046,11 +1068,11 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         int u, pp;
         decode_item(p, item, u, pp);
-        (void)u;
-        for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-          const int I = pass_block(p, pp, pass);
+        const Unit U = decode_unit(p, u);
+        for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+          const int I = pass_block(U, pp, pass);
           if (!(ok = mbar_wait_warp(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
-          const int nT = n_col_tiles64(p, I);
+          const int nT = n_col_tiles64(p, U, I);
           int prev_ts = -1;
           for (int J = 0; J < nT; ++J) {
             const int tt = nJ & 1, ts = nJ & 3, b = ns & 1;
@@ -1106,9 +1128,9 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
       int u, pp;
         decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
-      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-        const int I = pass_block(p, pp, pass);
-        const int nT = n_col_tiles64(p, I);
+      for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+        const int I = pass_block(U, pp, pass);
+        const int nT = n_col_tiles64(p, U, I);
         for (int J = 0; J < nT; ++J) {
           const int b = np & 1;
           ok = mbar_wait(P_FULL(b), (np >> 1) & 1, wc, W_EPI_P_FULL);
@@ -1137,7 +1159,7 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
                             v[jj]);
             fence_proxy_async_smem();
             __syncwarp();
-            const int row0 = J * BN64 + jb * 32;
+            const int row0 = U.tok0 + J * BN64 + jb * 32;
             if (lane == 0) {
               if (row0 < p.N) tma_reduce_add_4d(&U.seg->tm_dx, buf, q * 32, row0, U.h, U.b);
               bulk_commit();
@@ -1151,7 +1173,7 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        epilogue_reduce<D>(tmem + lane_addr + T_DXI, stg, nstg, &U.seg->tm_dx, I * BM + q * 32,
+        epilogue_reduce<D>(tmem + lane_addr + T_DXI, stg, nstg, &U.seg->tm_dx, U.tok0 + I * BM + q * 32,
                            U.h, U.b, p.N, lane, DXI_EMPTY);
         ++nrb;
       }
@@ -1171,10 +1193,10 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
       int u, pp;
         decode_item(p, item, u, pp);
       const Unit U = decode_unit(p, u);
-      for (int pass = 0; ok && pass < item_passes(p, pp); ++pass) {
-        const int I = pass_block(p, pp, pass);
+      for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
+        const int I = pass_block(U, pp, pass);
         const int row = I * BM + r;
-        const int L = unit_len(p, U);
+        const int L = U.len;
         const bool rvalid = row < L;
         float bt = 0.f, bs = 0.f, mul = 0.f;
         if (rvalid) {
@@ -1185,7 +1207,7 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
           mul = up * p.scale;   // the logit scale of dX_s is folded into G
         }
         const int lim = !rvalid ? -1 : (p.causal ? min(row, L - 1) : L - 1);
-        const int nT = n_col_tiles64(p, I);
+        const int nT = n_col_tiles64(p, U, I);
         const float2 sl2v = make_float2(sl2, sl2), btv = make_float2(bt, bt),
                      bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
                      m1 = make_float2(-1.f, -1.f);
@@ -1298,8 +1320,9 @@ constexpr int kPairMinBlocks = 33;
 constexpr int BWDP_LOGIT_WARP = 21, BWDP_GRAD_WARP = 22;
 
 // Sequence `which` (0 or 1) of pair item m: its first row block, or -1.
-__device__ __forceinline__ int pair_seq_block(const TcParams& p, int m, int which) {
-  const int npb = (p.nblk + 1) / 2;
+__device__ __forceinline__ int pair_seq_block(const Unit& U, int m, int which) {
+  const int npb = (U.nblk + 1) / 2;
+  if (m >= (npb + 1) / 2) return -1;   // past a short packed sequence's items
   const int k = which == 0 ? npb - 1 - m : m;
   if (which == 1 && k == npb - 1 - m) return -1;
   return 2 * k;
@@ -1385,24 +1408,24 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         decode_item(p, item, u, m);
         const Unit U = decode_unit(p, u);
         for (int w = 0; ok && w < 2; ++w) {
-          const int R0 = pair_seq_block(p, m, w);
+          const int R0 = pair_seq_block(U, m, w);
           if (R0 < 0) break;
-          const bool has1 = R0 + 1 < p.nblk;
+          const bool has1 = R0 + 1 < U.nblk;
           if (!(ok = mbar_wait(EMPTY_I, (nseq & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
           mbar_arrive_expect_tx(FULL_I, (has1 ? 4 : 2) * L::TILE_I);
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
-            tma_load_4d(base + L::XT_R0 + b * L::BOX_I, &U.seg->tm_t, FULL_I, b * 64, R0 * BM, U.h, U.b);
-            tma_load_4d(base + L::XS_R0 + b * L::BOX_I, &U.seg->tm_s, FULL_I, b * 64, R0 * BM, U.h, U.b);
+            tma_load_4d(base + L::XT_R0 + b * L::BOX_I, &U.seg->tm_t, FULL_I, b * 64, U.tok0 + R0 * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_R0 + b * L::BOX_I, &U.seg->tm_s, FULL_I, b * 64, U.tok0 + R0 * BM, U.h, U.b);
             if (has1) {
-              tma_load_4d(base + L::XT_R1 + b * L::BOX_I, &U.seg->tm_t, FULL_I, b * 64, (R0 + 1) * BM,
+              tma_load_4d(base + L::XT_R1 + b * L::BOX_I, &U.seg->tm_t, FULL_I, b * 64, U.tok0 + (R0 + 1) * BM,
                           U.h, U.b);
-              tma_load_4d(base + L::XS_R1 + b * L::BOX_I, &U.seg->tm_s, FULL_I, b * 64, (R0 + 1) * BM,
+              tma_load_4d(base + L::XS_R1 + b * L::BOX_I, &U.seg->tm_s, FULL_I, b * 64, U.tok0 + (R0 + 1) * BM,
                           U.h, U.b);
             }
           }
           ++nseq;
-          const int nT = n_col_tiles64(p, has1 ? R0 + 1 : R0);
+          const int nT = n_col_tiles64(p, U, has1 ? R0 + 1 : R0);
           for (int J = 0; J < nT; ++J) {
             const int tt = nJ & 1, ts = nJ & 1;
             if (!(ok = mbar_wait(EMPTY_T(tt), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
@@ -1410,14 +1433,14 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
             for (int b = 0; b < 2; ++b)
               tma_load_4d(base + L::XT_J + tt * L::TILE_J + b * L::BOX_J, &U.seg->tm_t64, FULL_T(tt),
-                          b * 64, J * BN64, U.h, U.b);
+                          b * 64, U.tok0 + J * BN64, U.h, U.b);
             ++armsT[tt];
             if (!(ok = mbar_wait(EMPTY_S(ts), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
             mbar_arrive_expect_tx(FULL_S(ts), L::TILE_J);
 #pragma unroll
             for (int b = 0; b < 2; ++b)
               tma_load_4d(base + L::XS_J + ts * L::TILE_J + b * L::BOX_J, &U.seg->tm_s64, FULL_S(ts),
-                          b * 64, J * BN64, U.h, U.b);
+                          b * 64, U.tok0 + J * BN64, U.h, U.b);
             ++armsS[ts];
             ++nJ;
           }
@@ -1458,13 +1481,13 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
       int u, m;
       decode_item(p, item, u, m);
-      (void)u;
+      const Unit U = decode_unit(p, u);
       for (int w = 0; ok && w < 2; ++w) {
-        const int R0 = pair_seq_block(p, m, w);
+        const int R0 = pair_seq_block(U, m, w);
         if (R0 < 0) break;
-        const bool has1 = R0 + 1 < p.nblk;
-        const int nT0 = n_col_tiles64(p, R0);
-        const int nT = has1 ? n_col_tiles64(p, R0 + 1) : nT0;
+        const bool has1 = R0 + 1 < U.nblk;
+        const int nT0 = n_col_tiles64(p, U, R0);
+        const int nT = has1 ? n_col_tiles64(p, U, R0 + 1) : nT0;
         if (!(ok = mbar_wait_warp(FULL_I, nseq & 1, wc, W_MMA_FULL_I))) break;
         bool first_seq = true;
         for (int J = 0; ok && J < nT; ++J) {
@@ -1560,10 +1583,10 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         decode_item(p, item, u, m);
       const Unit U = decode_unit(p, u);
       for (int w = 0; ok && w < 2; ++w) {
-        const int R0 = pair_seq_block(p, m, w);
+        const int R0 = pair_seq_block(U, m, w);
         if (R0 < 0) break;
-        const bool has1 = R0 + 1 < p.nblk;
-        const int nT = n_col_tiles64(p, has1 ? R0 + 1 : R0);
+        const bool has1 = R0 + 1 < U.nblk;
+        const int nT = n_col_tiles64(p, U, has1 ? R0 + 1 : R0);
         for (int J = 0; J < nT; ++J) {
           const int b = np & 1;
           ok = mbar_wait(P_FULL(b), (np >> 1) & 1, wc, W_EPI_P_FULL);
@@ -1587,7 +1610,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
               st_shared_b32(stg + jj * 128 + (((lane >> 2) ^ (jj & 7)) << 4) + (lane & 3) * 4, v[jj]);
             fence_proxy_async_smem();
             __syncwarp();
-            const int row0 = J * BN64 + jb * 32;
+            const int row0 = U.tok0 + J * BN64 + jb * 32;
             if (lane == 0) {
               if (row0 < p.N) tma_reduce_add_4d(&U.seg->tm_dx, stg, q * 32, row0, U.h, U.b);
               bulk_commit();
@@ -1602,7 +1625,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         if (!ok) break;
         tc_fence_after();
         for (int rs = 0; rs < 2; ++rs) {
-          const int row0 = (R0 + rs) * BM + q * 32;
+          const int row0 = U.tok0 + (R0 + rs) * BM + q * 32;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             float v[32];
@@ -1649,12 +1672,12 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         decode_item(p, item, u, m);
       const Unit U = decode_unit(p, u);
       for (int w = 0; ok && w < 2; ++w) {
-        const int R0 = pair_seq_block(p, m, w);
+        const int R0 = pair_seq_block(U, m, w);
         if (R0 < 0) break;
-        const bool has1 = R0 + 1 < p.nblk;
-        const int nT0 = n_col_tiles64(p, R0);
-        const int nT = has1 ? n_col_tiles64(p, R0 + 1) : nT0;
-        const int L = unit_len(p, U);
+        const bool has1 = R0 + 1 < U.nblk;
+        const int nT0 = n_col_tiles64(p, U, R0);
+        const int nT = has1 ? n_col_tiles64(p, U, R0 + 1) : nT0;
+        const int L = U.len;
         // per-row constants of both row blocks
         float bt[2], bs[2], mul[2];
         int lim[2];

@@ -37,8 +37,25 @@ def _lengths_ptr(lengths: Optional[torch.Tensor], x: torch.Tensor) -> Optional[i
     return int(lengths.data_ptr())
 
 
+def _cu_ptr(cu_seqlens: Optional[torch.Tensor], x: torch.Tensor) -> Optional[int]:
+    """Device pointer of packed-sequence offsets (int32 [n_seq + 1] on x's device), or None."""
+    if cu_seqlens is None:
+        return None
+    if (cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1
+            or not cu_seqlens.is_contiguous() or cu_seqlens.device != x.device):
+        raise ValueError("cu_seqlens must be a contiguous int32 [n_seq + 1] tensor on the "
+                         "inputs' device")
+    if x.shape[0] != 1:
+        raise ValueError("packed sequences use [1, H, N, d] tensors")
+    return int(cu_seqlens.data_ptr())
+
+
 def make_desc(x: torch.Tensor, causal: bool = True, scale: float = 0.0,
-              lengths: Optional[torch.Tensor] = None) -> relkl_desc:
+              lengths: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
+              max_seqlen: int = 0) -> relkl_desc:
+    """C descriptor of a [B, H, N, d] tensor.  ``cu_seqlens`` (int32 [n_seq + 1],
+    device) makes it packed sequences on one token axis, B = 1; ``max_seqlen``
+    must then bound every sequence's length."""
     if x.dim() != 4:
         raise ValueError("expected a [B, H, N, d] tensor")
     if x.dtype not in _DTYPES:
@@ -53,6 +70,11 @@ def make_desc(x: torch.Tensor, causal: bool = True, scale: float = 0.0,
     d.scale = float(scale)
     d.reserved = 0
     d.lengths = _lengths_ptr(lengths, x)
+    d.cu_seqlens = _cu_ptr(cu_seqlens, x)
+    d.n_seq = 0 if cu_seqlens is None else int(cu_seqlens.numel()) - 1
+    d.max_seqlen = 0 if cu_seqlens is None else int(max_seqlen)
+    if cu_seqlens is not None and not 0 <= d.max_seqlen <= d.N:
+        raise ValueError("max_seqlen must lie in [0, N]")
     return d
 
 
@@ -128,8 +150,11 @@ def _part(part) -> Tuple[int, int]:
 def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bool = True,
                   scale: float = 0.0, *, out: Optional[Sequence[Tuple[torch.Tensor, torch.Tensor]]] = None,
                   ws: Optional[torch.Tensor] = None, stream=None,
-                  lengths: Optional[torch.Tensor] = None, part=None):
+                  lengths: Optional[torch.Tensor] = None, part=None,
+                  cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: int = 0):
     """Forward over 1..3 relations in one launch.  Returns [(kl, stats)] per relation.
+    ``cu_seqlens``/``max_seqlen``: packed sequences on one token axis ([1, H, N, d]
+    tensors; see relkl_desc), shared by the relations.
     ``lengths``: optional int32 [B] valid lengths (right padding), shared by the relations.
     ``part``: (index, count) to compute only that part of every unit's rows
     (relkl_fwd_qkv_part); outputs allocated here are then zero elsewhere."""
@@ -145,7 +170,7 @@ def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bo
         _cuda(xs, "x_s")
         if xt.shape != xs.shape or xt.stride() != xs.stride() or xt.dtype != xs.dtype:
             raise ValueError("teacher and student must share shape, strides and dtype")
-        descs[r] = make_desc(xt, causal, scale, lengths)
+        descs[r] = make_desc(xt, causal, scale, lengths, cu_seqlens, max_seqlen)
         B, H, N, _ = xt.shape
         if xt.device != dev or xs.device != dev:
             raise ValueError("every relation must live on the same device")
@@ -154,7 +179,9 @@ def relkl_fwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], causal: bo
             _check_out(kl, (B, H, N), "kl", dev)
             _check_out(st, (B, H, N, 4), "stats", dev)
         else:
-            alloc = torch.empty if n_parts == 1 else torch.zeros
+            # rows a call may leave untouched (other parts, tokens past the
+            # last packed sequence) come back as zeros
+            alloc = torch.empty if (n_parts == 1 and cu_seqlens is None) else torch.zeros
             kl = alloc((B, H, N), dtype=torch.float32, device=dev)
             st = alloc((B, H, N, 4), dtype=torch.float32, device=dev)
         outs.append((kl, st))
@@ -175,7 +202,9 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
                   dkl: Optional[Sequence[Optional[torch.Tensor]]] = None, causal: bool = True,
                   scale: float = 0.0, *, out: Optional[Sequence[torch.Tensor]] = None,
                   ws: Optional[torch.Tensor] = None, stream=None,
-                  lengths: Optional[torch.Tensor] = None, part=None) -> List[torch.Tensor]:
+                  lengths: Optional[torch.Tensor] = None, part=None,
+                  cu_seqlens: Optional[torch.Tensor] = None,
+                  max_seqlen: int = 0) -> List[torch.Tensor]:
     """Backward over 1..3 relations in one launch.  Returns dX_s per relation (float32).
     ``part``: (index, count) to return only that part's rows' contribution to
     dX_s (relkl_bwd_qkv_part); ``stats`` must then hold every row."""
@@ -193,7 +222,7 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
             raise ValueError("teacher and student must share shape, strides and dtype")
         if xt.device != dev or xs.device != dev:
             raise ValueError("every relation must live on the same device")
-        descs[r] = make_desc(xt, causal, scale, lengths)
+        descs[r] = make_desc(xt, causal, scale, lengths, cu_seqlens, max_seqlen)
         B, H, N, _ = xt.shape
         _check_out(stats[r], (B, H, N, 4), "stats", dev)
         if dkl is not None and dkl[r] is not None:
@@ -218,24 +247,26 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
 def relkl_fwd(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True, scale: float = 0.0, *,
               kl: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
               ws: Optional[torch.Tensor] = None, stream=None,
-              lengths: Optional[torch.Tensor] = None):
+              lengths: Optional[torch.Tensor] = None,
+              cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: int = 0):
     """Per-row KL [B,H,N] and statistics [B,H,N,4] of one relation.  Pass both
     ``kl`` and ``stats`` to write into existing tensors, or neither."""
     if (kl is None) != (stats is None):
         raise ValueError("pass both kl and stats, or neither")
     out = None if kl is None else [(kl, stats)]
     return relkl_fwd_qkv([(x_t, x_s)], causal, scale, out=out, ws=ws, stream=stream,
-                         lengths=lengths)[0]
+                         lengths=lengths, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)[0]
 
 
 def relkl_bwd(x_t: torch.Tensor, x_s: torch.Tensor, stats: torch.Tensor,
               dkl: Optional[torch.Tensor] = None, causal: bool = True, scale: float = 0.0, *,
               dx_s: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
-              stream=None, lengths: Optional[torch.Tensor] = None) -> torch.Tensor:
+              stream=None, lengths: Optional[torch.Tensor] = None,
+              cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: int = 0) -> torch.Tensor:
     """dL/dX_s (float32) with L = sum_i dkl_i kl_i (dkl=None: 1/N per row, 1/L_b with lengths)."""
     return relkl_bwd_qkv([(x_t, x_s)], [stats], None if dkl is None else [dkl], causal, scale,
                          out=None if dx_s is None else [dx_s], ws=ws, stream=stream,
-                         lengths=lengths)[0]
+                         lengths=lengths, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)[0]
 
 
 def relkl_fwd_noalloc(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,

@@ -81,6 +81,21 @@ typedef struct {
    * a valid row is 1/L_b.  Read on the device; must stay valid until the
    * queued work has finished; 4-byte aligned.                               */
   const int32_t* lengths;
+  /* Optional packed variable-length sequences (cu_seqlens NULL: none).  The
+   * tensors are [1, H, N, d] (B must be 1, lengths NULL) and hold n_seq
+   * sequences back to back on the token axis: sequence k owns tokens
+   * [cu_seqlens[k], cu_seqlens[k+1]) (DEVICE int32 [n_seq + 1],
+   * non-decreasing, cu_seqlens[0] = 0, cu_seqlens[n_seq] <= N; read on the
+   * device, 4-byte aligned).  Each (sequence, head) is a unit of its own: its
+   * rows see only its own tokens (causal or full inside it), its default
+   * upstream gradient is 1/L_k, and kl, stats and dX_s use the [1, H, N]
+   * layout of the tokens.  Tokens past cu_seqlens[n_seq] belong to no
+   * sequence: the forward leaves their kl and stats rows untouched and their
+   * dX_s rows are 0.  max_seqlen must be >= every sequence's length (it sizes
+   * the work; rows of a longer sequence past max_seqlen are not computed).  */
+  const int32_t* cu_seqlens;
+  int32_t n_seq;
+  int32_t max_seqlen;
 } relkl_desc;
 
 /* Bytes of device workspace a call needs (for every entry point, any desc):

@@ -46,7 +46,8 @@ import numpy as np
 import torch
 
 __all__ = ["as_f64", "relation_logits", "allowed", "fwd_unit", "bwd_unit",
-           "fwd_rows", "bwd_rows", "fwd", "bwd", "unit_loss", "relation_probs", "bwd_contrib"]
+           "fwd_rows", "bwd_rows", "fwd", "bwd", "unit_loss", "relation_probs", "bwd_contrib",
+           "fwd_varlen", "bwd_varlen"]
 
 
 def as_f64(x) -> np.ndarray:
@@ -270,4 +271,50 @@ def bwd_contrib(xt, xs, rows: Iterable[int], dkl=None, causal: bool = True,
     g = g_up[rows, None] * np.where(ok, np.exp(logp_s) - np.exp(logp_t), 0.0)
     dx[rows] += s * (g @ xs)              # row side
     dx += s * (g.T @ xs[rows])            # column side
+    return dx
+
+
+def _seq_bounds(cu_seqlens, N: int):
+    cu = np.asarray(cu_seqlens, dtype=np.int64).reshape(-1)
+    if cu.size < 1 or cu[0] != 0 or np.any(np.diff(cu) < 0) or cu[-1] > N:
+        raise ValueError("cu_seqlens must start at 0, not decrease and end at most at N")
+    return cu
+
+
+def fwd_varlen(xt, xs, cu_seqlens, causal: bool = True, scale: Optional[float] = None,
+               slab: int = 2048) -> Dict[str, np.ndarray]:
+    """Packed variable-length sequences: [1, H, N, d] holds sequences back to
+    back on one token axis, sequence k on tokens [cu[k], cu[k+1]).  Each
+    sequence is its own relation: its rows see only its own tokens (masked as
+    usual inside it).  Statistics come back as [1, H, N]; tokens past the last
+    sequence stay 0."""
+    xt, xs = as_f64(xt), as_f64(xs)
+    _, H, N, _ = xt.shape
+    cu = _seq_bounds(cu_seqlens, N)
+    out = {k: np.zeros((1, H, N)) for k in ("kl", "lse_t", "lse_s", "w", "m")}
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b == a:
+            continue
+        for h in range(H):
+            r = fwd_unit(xt[0, h, a:b], xs[0, h, a:b], causal, scale, slab)
+            for k in out:
+                out[k][0, h, a:b] = r[k]
+    return out
+
+
+def bwd_varlen(xt, xs, cu_seqlens, dkl=None, causal: bool = True,
+               scale: Optional[float] = None, slab: int = 2048) -> np.ndarray:
+    """dL/dX_s of packed sequences; ``dkl`` is [1, H, N] or None (1/L_k on every
+    row of a sequence of length L_k).  Tokens past the last sequence get 0."""
+    xt, xs = as_f64(xt), as_f64(xs)
+    _, H, N, _ = xt.shape
+    cu = _seq_bounds(cu_seqlens, N)
+    g = None if dkl is None else as_f64(dkl).reshape(1, H, N)
+    dx = np.zeros_like(xs)
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b == a:
+            continue
+        for h in range(H):
+            dx[0, h, a:b] = bwd_unit(xt[0, h, a:b], xs[0, h, a:b],
+                                     None if g is None else g[0, h, a:b], causal, scale, slab)
     return dx

@@ -410,3 +410,55 @@ def test_row_partition_contributions_sum_to_the_gradient(causal):
     want = np.outer(g_i, xs[i]) * s
     want[i] += s * (g_i @ xs)
     np.testing.assert_allclose(one, want, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_packed_sequences_equal_separate_batches(causal):
+    """Packed sequences of equal length L are a batch [n_seq, H, L, d] laid on one
+    token axis: the packed oracle must equal the batched one on the reshaped
+    tensors (pins the packing's index arithmetic), and a sequence must not see
+    its neighbours (changing one sequence leaves the others' rows unchanged)."""
+    n_seq, H, L, d = 3, 2, 9, 4
+    xt, xs = workload.gaussian_pair((n_seq, H, L, d), seed=61, noise=0.5, dtype=torch.float64)
+    packed_t = xt.permute(1, 0, 2, 3).reshape(1, H, n_seq * L, d)
+    packed_s = xs.permute(1, 0, 2, 3).reshape(1, H, n_seq * L, d)
+    cu = [0, L, 2 * L, 3 * L]
+    dkl = torch.linspace(-1.0, 1.0, n_seq * H * L, dtype=torch.float64).reshape(n_seq, H, L)
+    dkl_packed = dkl.permute(1, 0, 2).reshape(1, H, n_seq * L)
+    ref = dense.fwd(xt, xs, causal)
+    got = dense.fwd_varlen(packed_t, packed_s, cu, causal)
+    for k in ("kl", "lse_t", "lse_s", "w", "m"):
+        np.testing.assert_allclose(got[k].reshape(H, n_seq, L).transpose(1, 0, 2), ref[k],
+                                   rtol=1e-13, atol=1e-15)
+    ref_dx = dense.bwd(xt, xs, dkl, causal)
+    got_dx = dense.bwd_varlen(packed_t, packed_s, cu, dkl_packed, causal)
+    np.testing.assert_allclose(got_dx.reshape(H, n_seq, L, d).transpose(1, 0, 2, 3), ref_dx,
+                               rtol=1e-12, atol=1e-15)
+    # default upstream gradient: 1/L per row of each sequence
+    np.testing.assert_allclose(dense.bwd_varlen(packed_t, packed_s, cu, None, causal)
+                               .reshape(H, n_seq, L, d).transpose(1, 0, 2, 3),
+                               dense.bwd(xt, xs, None, causal), rtol=1e-12, atol=1e-15)
+    # isolation: perturb sequence 1 only
+    pt2 = packed_t.clone()
+    pt2[:, :, L:2 * L] += 1.0
+    other = dense.fwd_varlen(pt2, packed_s, cu, causal)["kl"]
+    np.testing.assert_array_equal(other[:, :, :L], got["kl"][:, :, :L])
+    np.testing.assert_array_equal(other[:, :, 2 * L:], got["kl"][:, :, 2 * L:])
+    assert np.abs(other[:, :, L:2 * L] - got["kl"][:, :, L:2 * L]).max() > 1e-3
+
+
+def test_packed_sequences_ragged_and_empty():
+    """Unequal lengths, an empty sequence and tokens past the last sequence."""
+    H, N, d = 1, 30, 4
+    xt, xs = workload.gaussian_pair((1, H, N, d), seed=62, noise=0.5, dtype=torch.float64)
+    cu = [0, 7, 7, 20, 26]
+    got = dense.fwd_varlen(xt, xs, cu)
+    for a, b in ((0, 7), (7, 20), (20, 26)):
+        np.testing.assert_allclose(got["kl"][0, 0, a:b], dense.fwd_unit(xt[0, 0, a:b],
+                                                                        xs[0, 0, a:b])["kl"],
+                                   rtol=1e-13, atol=1e-15)
+    assert np.all(got["kl"][0, 0, 26:] == 0)
+    dx = dense.bwd_varlen(xt, xs, cu)
+    assert np.all(dx[0, 0, 26:] == 0)
+    with pytest.raises(ValueError):
+        dense.fwd_varlen(xt, xs, [0, 5, 3])
