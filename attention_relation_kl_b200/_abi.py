@@ -85,7 +85,8 @@ def _declare(lib):
     lib.relkl_rope_bwd.restype = ctypes.c_int
     lib.relkl_rope_bwd.argtypes = [i32, i32, i32, i32, _vp, ctypes.POINTER(relkl_rope), i32, _vp, _vp]
     lib.relkl_weight_grad.restype = ctypes.c_int
-    lib.relkl_weight_grad.argtypes = [ctypes.c_int64, i32, i32, _vp, _vp, _vp, _vp]
+    lib.relkl_weight_grad.argtypes = [ctypes.c_int64, i32, i32, _vp, _vp, _vp, _vp,
+                                      ctypes.c_size_t, _vp]
     return lib
 
 
@@ -107,7 +108,7 @@ class RelklError(RuntimeError):
     def __init__(self, code: int, where: str):
         msg = lib().relkl_status_string(code).decode()
         if code == RELKL_ERR_CUDA:
-            msg += f" (CUDA / cuBLAS status {lib().relkl_last_cuda_error()})"
+            msg += f" (CUDA status {lib().relkl_last_cuda_error()})"
         super().__init__(f"{where}: {msg}")
         self.code = code
 

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "librelkl.so")
-SOURCES = ["relkl_api.cu", "relkl_tc.cu", "relkl_simt.cu", "relkl_chain.cu"]
+SOURCES = ["relkl_api.cu", "relkl_tc.cu", "relkl_simt.cu", "relkl_chain.cu", "relkl_gemm.cu"]
 HEADERS = ["relkl_device.cuh", "relkl_params.h"]
 
 NVCC_FLAGS = [
@@ -50,7 +50,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + ".tmp"
     cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
-           *[os.path.join(CSRC, f) for f in SOURCES], "-lcublas", "-ldl", "-o", tmp]
+           *[os.path.join(CSRC, f) for f in SOURCES], "-ldl", "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)

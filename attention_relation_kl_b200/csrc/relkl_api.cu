@@ -25,8 +25,13 @@ cudaError_t launch_zero(float* ptr, int64_t n, int num_sms, cudaStream_t stream)
 cudaError_t launch_rope_bwd(const float* dx, void* out, int B, int H, int N, int d, bool bf16_out,
                             double base, double pos_scale, double pos_offset, int apply,
                             cudaStream_t stream);
-int chain_weight_grad(long long rows, int D, int cols, const void* h, const void* dx_pre,
-                      float* dw, cudaStream_t stream);
+using EncodeTiledFnG = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+int launch_wgrad(EncodeTiledFnG encode, long long rows, int D, int cols, const void* h,
+                 const void* dx_pre, float* dw, int num_sms, DevStatus* status,
+                 unsigned long long timeout_ns, cudaStream_t stream);
 }  // namespace relkl
 
 using namespace relkl;
@@ -538,17 +543,25 @@ relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const fl
 }
 
 relkl_status relkl_weight_grad(int64_t rows, int32_t D, int32_t cols, const void* h,
-                               const void* dx_pre, float* dw, void* stream) {
+                               const void* dx_pre, float* dw, void* ws, size_t ws_bytes,
+                               void* stream) {
   NvtxRange nvtx_range("relkl_weight_grad");
   if (rows < 1 || rows > 0x7fffffffLL || D < 1 || cols < 1 || (D % 8) || (cols % 8))
     return RELKL_ERR_INVALID;
   if (!h || !dx_pre || !dw || !aligned(h, 16) || !aligned(dx_pre, 16) || !aligned(dw, 16))
     return RELKL_ERR_INVALID;
-  const int st = chain_weight_grad(rows, D, cols, h, dx_pre, dw, static_cast<cudaStream_t>(stream));
-  if (st != 0) {
-    g_last_cuda = st;
-    return RELKL_ERR_CUDA;
-  }
+  relkl_status s = check_ws(ws, ws_bytes);
+  if (s != RELKL_OK) return s;
+  DevInfo dev;
+  if ((s = device_info(&dev)) != RELKL_OK) return s;
+  if (dev.major != 10) return RELKL_ERR_UNSUPPORTED;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return RELKL_ERR_CUDA;
+  const int r = launch_wgrad(enc, rows, D, cols, h, dx_pre, dw, dev.sms,
+                             reinterpret_cast<DevStatus*>(ws), g_timeout_ns.load(),
+                             static_cast<cudaStream_t>(stream));
+  if (r == 1) return RELKL_ERR_UNSUPPORTED;
+  if (r != 0) return cuda_fail(static_cast<cudaError_t>(r - 2));
   return RELKL_OK;
 }
 

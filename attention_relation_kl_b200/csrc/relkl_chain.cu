@@ -7,8 +7,8 @@
 //     rotation of the post-RoPE gradient (g_a cos + g_b sin, g_b cos - g_a sin).
 //     The kernel also moves heads next to each other per token
 //     ([B, H, N, d] -> [B, N, H, d]), the row layout of X = H_s W.
-//   * Weight gradient dW = H_s^T dX_pre over the B*N token rows: one plain
-//     GEMM, issued to cuBLAS (bf16 operands, fp32 accumulation and result).
+//   * Weight gradient dW = H_s^T dX_pre over the B*N token rows: the tcgen05
+//     GEMM in relkl_gemm.cu (bf16 operands, fp32 accumulation and result).
 //
 // LinearARD trains only the student's Q/K/V projections (pith.science
 // verdict page, ``minor_comments``); the pages stop at the logit gradient, so
@@ -17,7 +17,6 @@
 #include <cstdint>
 #include <mutex>
 
-#include <cublas_v2.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -161,40 +160,6 @@ cudaError_t launch_rope_bwd(const float* dx, void* out, int B, int H, int N, int
     rope_bwd_kernel<false><<<grid, block, 0, stream>>>(dx, out, H, N, d, lb, pos_scale, pos_offset,
                                                        apply);
   return cudaGetLastError();
-}
-
-// dW [D, cols] (row-major, fp32) = H^T dX_pre with H [rows, D] and dX_pre
-// [rows, cols] row-major bf16.  In cuBLAS's column-major terms that is
-// C [cols x D] = A [cols x rows] * B [rows x D] with A the memory of dX_pre
-// (no transpose) and B the transpose of the memory of H.  One handle per
-// device, created on first use without a workspace (cuBLAS then picks
-// algorithms that need none); calls are serialised on it.
-int chain_weight_grad(long long rows, int D, int cols, const void* h, const void* dx_pre,
-                      float* dw, cudaStream_t stream) {
-  static std::mutex mu;
-  static cublasHandle_t handles[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-    return static_cast<int>(CUBLAS_STATUS_NOT_INITIALIZED);
-  std::lock_guard<std::mutex> lk(mu);
-  if (!handles[dev]) {
-    cublasHandle_t hd = nullptr;
-    cublasStatus_t st = cublasCreate(&hd);
-    if (st != CUBLAS_STATUS_SUCCESS) return static_cast<int>(st);
-    if ((st = cublasSetWorkspace(hd, nullptr, 0)) != CUBLAS_STATUS_SUCCESS) {
-      cublasDestroy(hd);
-      return static_cast<int>(st);
-    }
-    handles[dev] = hd;
-  }
-  cublasHandle_t hd = handles[dev];
-  cublasStatus_t st = cublasSetStream(hd, stream);
-  if (st != CUBLAS_STATUS_SUCCESS) return static_cast<int>(st);
-  const float alpha = 1.0f, beta = 0.0f;
-  st = cublasGemmEx(hd, CUBLAS_OP_N, CUBLAS_OP_T, cols, D, static_cast<int>(rows), &alpha, dx_pre,
-                    CUDA_R_16BF, cols, h, CUDA_R_16BF, D, &beta, dw, CUDA_R_32F, cols,
-                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-  return static_cast<int>(st);
 }
 
 }  // namespace relkl

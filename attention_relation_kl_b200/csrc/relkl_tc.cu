@@ -892,6 +892,86 @@ static_assert(Bwd64Smem::ALLOC <= 232448, "backward shared memory exceeds 227 KB
 
 constexpr int BN64 = 64;
 
+// Column tiles of row block I in the paired-block kernels.  With SYM (full
+// masks) only the tiles up to the diagonal block are visited, as under the
+// causal mask: each off-diagonal tile then serves both orientations of its
+// entries (Z = Z^T).
+template <bool SYM>
+__device__ __forceinline__ int n_col_tiles64_s(const TcParams& p, const Unit& U, int I) {
+  const int nb64 = (U.span + BN64 - 1) / BN64;
+  return (p.causal || SYM) ? min(2 * I + 2, nb64) : nb64;
+}
+template <bool SYM>
+__device__ __forceinline__ int n_col_tiles_s(const TcParams& p, const Unit& U, int I) {
+  return (p.causal || SYM) ? I + 1 : U.nblk;
+}
+
+// Row-side G plus, for an entry (i, j) off the diagonal block of a full mask,
+// its transposed partner G(j, i) = dkl_j (R_s - R_t)(j, i), which reuses the
+// logits because Z(j, i) = Z(i, j).  Row j's LSEs and upstream gradient come
+// from the statistics of column j.  Adds the partners of columns c, c+1
+// (local to the unit) to g; zt2 / zs2 are the raw logit accumulators of the
+// pair.
+__device__ __forceinline__ float2 sym_partner(const Unit& U, const TcParams& p, int c, float2 zt2,
+                                              float2 zs2, float2 g) {
+  // keep this pair's loads next to their use: hoisting all of a tile's column
+  // statistics ahead of the exps would not fit the row warps' registers
+  __syncwarp();
+  const float4* st = reinterpret_cast<const float4*>(U.seg->stats) + U.row0;
+  const int last = U.span - 1;
+  const int c0 = min(c, last), c1 = min(c + 1, last);
+  const float4 a = st[c0], b = st[c1];
+  const float2 btc = make_float2(-a.y * kLog2e, -b.y * kLog2e);
+  const float2 bsc = make_float2(-a.z * kLog2e, -b.z * kLog2e);
+  float2 mulc;
+  if (U.seg->dkl) {
+    const float* dk = U.seg->dkl + U.row0;
+    mulc = make_float2(dk[c0] * p.scale, dk[c1] * p.scale);
+  } else {
+    const float m = p.scale / static_cast<float>(U.len);
+    mulc = make_float2(m, m);
+  }
+  const float2 sl2v = make_float2(p.sl2, p.sl2);
+  const float2 et = ex2_approx2(__ffma2_rn(zt2, sl2v, btc));
+  const float2 es = ex2_approx2(__ffma2_rn(zs2, sl2v, bsc));
+  return __ffma2_rn(__ffma2_rn(et, make_float2(-1.f, -1.f), es), mulc, g);
+}
+
+// Forms NC consecutive entries of one row of the bf16 gradient tile and
+// stores them as NC/8 16-byte chunks (chunk0, chunk0 + 1, ...) of the row's
+// 128-byte swizzled line at row_addr.  bt, bs: -lse * log2 e of the row;
+// mul: its upstream gradient times the logit scale; entries past `lim` are 0;
+// `off`: add the transposed partner (full mask, off the diagonal block).
+template <int NC>
+__device__ __forceinline__ void form_g_store(const float (&t)[NC], const float (&s)[NC],
+                                             float bt, float bs, float mul, int col0, int lim,
+                                             bool off, const Unit& U, const TcParams& p,
+                                             uint32_t row_addr, int chunk0, int r) {
+  const float2 sl2v = make_float2(p.sl2, p.sl2), btv = make_float2(bt, bt),
+               bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
+               m1 = make_float2(-1.f, -1.f);
+  const bool need_mask = col0 + NC - 1 > lim;
+#pragma unroll
+  for (int q = 0; q < NC / 8; ++q) {
+    uint32_t pk[4];
+#pragma unroll
+    for (int k2 = 0; k2 < 8; k2 += 2) {
+      const int k = q * 8 + k2;
+      const float2 zt2 = make_float2(t[k], t[k + 1]), zs2 = make_float2(s[k], s[k + 1]);
+      const float2 et = ex2_approx2(__ffma2_rn(zt2, sl2v, btv));
+      const float2 es = ex2_approx2(__ffma2_rn(zs2, sl2v, bsv));
+      float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
+      if (off) g = sym_partner(U, p, col0 + k, zt2, zs2, g);
+      if (need_mask) {
+        g.x = (col0 + k <= lim) ? g.x : 0.f;
+        g.y = (col0 + k + 1 <= lim) ? g.y : 0.f;
+      }
+      pk[k2 >> 1] = pack_bf16x2(g.x, g.y);
+    }
+    st_shared_v4(row_addr + (((chunk0 + q) ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
 __device__ __forceinline__ int n_col_tiles64(const TcParams& p, const Unit& U, int I) {
   const int nb64 = (U.span + BN64 - 1) / BN64;
   return p.causal ? min(2 * I + 2, nb64) : nb64;
@@ -1328,6 +1408,7 @@ __device__ __forceinline__ int pair_seq_block(const Unit& U, int m, int which) {
   return 2 * k;
 }
 
+template <bool SYM>
 __global__ void __launch_bounds__(BWDP_THREADS, 1)
 relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
   using L = BwdPairSmem;
@@ -1425,7 +1506,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
             }
           }
           ++nseq;
-          const int nT = n_col_tiles64(p, U, has1 ? R0 + 1 : R0);
+          const int nT = n_col_tiles64_s<SYM>(p, U, has1 ? R0 + 1 : R0);
           for (int J = 0; J < nT; ++J) {
             const int tt = nJ & 1, ts = nJ & 1;
             if (!(ok = mbar_wait(EMPTY_T(tt), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
@@ -1486,8 +1567,8 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         const int R0 = pair_seq_block(U, m, w);
         if (R0 < 0) break;
         const bool has1 = R0 + 1 < U.nblk;
-        const int nT0 = n_col_tiles64(p, U, R0);
-        const int nT = has1 ? n_col_tiles64(p, U, R0 + 1) : nT0;
+        const int nT0 = n_col_tiles64_s<SYM>(p, U, R0);
+        const int nT = has1 ? n_col_tiles64_s<SYM>(p, U, R0 + 1) : nT0;
         if (!(ok = mbar_wait_warp(FULL_I, nseq & 1, wc, W_MMA_FULL_I))) break;
         bool first_seq = true;
         for (int J = 0; ok && J < nT; ++J) {
@@ -1586,7 +1667,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         const int R0 = pair_seq_block(U, m, w);
         if (R0 < 0) break;
         const bool has1 = R0 + 1 < U.nblk;
-        const int nT = n_col_tiles64(p, U, has1 ? R0 + 1 : R0);
+        const int nT = n_col_tiles64_s<SYM>(p, U, has1 ? R0 + 1 : R0);
         for (int J = 0; J < nT; ++J) {
           const int b = np & 1;
           ok = mbar_wait(P_FULL(b), (np >> 1) & 1, wc, W_EPI_P_FULL);
@@ -1675,8 +1756,8 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         const int R0 = pair_seq_block(U, m, w);
         if (R0 < 0) break;
         const bool has1 = R0 + 1 < U.nblk;
-        const int nT0 = n_col_tiles64(p, U, R0);
-        const int nT = has1 ? n_col_tiles64(p, U, R0 + 1) : nT0;
+        const int nT0 = n_col_tiles64_s<SYM>(p, U, R0);
+        const int nT = has1 ? n_col_tiles64_s<SYM>(p, U, R0 + 1) : nT0;
         const int L = U.len;
         // per-row constants of both row blocks
         float bt[2], bs[2], mul[2];
@@ -1718,6 +1799,16 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
             const float2 btv = make_float2(btr, btr), bsv = make_float2(bsr, bsr),
                          mulv = make_float2(mr, mr);
             const int col0 = J * BN64 + wg * 16;
+            if constexpr (SYM) {
+              // full mask: tiles of the diagonal block carry G itself, the others
+              // G plus its transposed partner (4 exps per entry: the exps bound
+              // this mode, so wait for the G buffer first and store as formed)
+              ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
+              ok = __all_sync(0xffffffffu, ok);
+              if (!ok) break;
+              form_g_store<16>(t, s, btr, bsr, mr, col0, limr, J < 2 * (R0 + rs), U, p, gsm,
+                               2 * wg, r);
+            } else {
             const bool need_mask = col0 + 15 > limr;
             uint32_t pk[8];
 #pragma unroll
@@ -1741,6 +1832,486 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
               const int cc = 2 * wg + h2;  // 16-byte chunk within the 128-byte row
               st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[4 * h2], pk[4 * h2 + 1], pk[4 * h2 + 2],
                            pk[4 * h2 + 3]);
+            }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(G_FULL);
+            ++nt;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == BWDP_LOGIT_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// =========================================================================
+//        BACKWARD, d = 64: adjacent row-block pairs, 128-column tiles
+// =========================================================================
+// The paired-block schedule of relkl_bwd_pair_kernel at head dimension 64.
+// The accumulators are half as wide as at d = 128, which leaves TMEM room for
+// 128-column logit tiles (full-rate N = 128 logit MMAs).  The column-side
+// product is formed as P = G^T X_s[R] (M = 128 columns j, N = d = 64,
+// K = the rows of R0 then R1), so it is summed over both row blocks in TMEM
+// and its TMEM lanes are the rows j of dX[J]: the epilogue stages them row by
+// row, without a transpose.  With 64-dimensional rows the exp work per entry
+// is what bounds this kernel (2 ex2 per entry against 0.08 clk of MMA work),
+// so one logit buffer and one G buffer suffice: the next tile's logit MMAs
+// and the previous tile's gradient MMAs finish while the row warps run the
+// current tile's exps.
+//   TMEM: Z_t 0..127, Z_s 128..255, dX_R0 256..319, dX_R1 320..383,
+//         P 2 x 64 at 384.
+//   smem: X_t, X_s of R0 and R1 (4 x 16 KB); teacher and student column
+//         rings 2 x 16 KB each; G 32 KB (two 64-column boxes); epilogue
+//         staging 4 x 4 KB.
+struct BwdPair64Smem {
+  static constexpr int TILE = BM * 64 * 2;           // 128 rows x 64 bf16: one box (16 KB)
+  static constexpr int XT_R0 = 0;
+  static constexpr int XS_R0 = TILE;
+  static constexpr int XT_R1 = 2 * TILE;
+  static constexpr int XS_R1 = 3 * TILE;
+  static constexpr int XT_J = 4 * TILE;              // 2 stages
+  static constexpr int XS_J = XT_J + 2 * TILE;       // 2 stages
+  static constexpr int G = XS_J + 2 * TILE;          // 128 x 128 bf16, boxes of 64 columns
+  static constexpr int STG = G + 2 * TILE;           // 4 warps x one 32 x 32 f32 box
+  static constexpr int STG_BYTES = 32 * 32 * 4;
+  static constexpr int BARS = STG + 4 * STG_BYTES;
+  // full_I, empty_I, fullT[2], emptyT[2], fullS[2], emptyS[2], s_full, s_empty,
+  // g_full, g_empty, p_full[2], p_empty[2], dxi_full, dxi_empty, drain x 2
+  static constexpr int NBAR = 22;
+  static constexpr int MISC = BARS + NBAR * 8;
+  static constexpr int BYTES = MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+};
+static_assert(BwdPair64Smem::ALLOC <= 232448, "backward shared memory exceeds 227 KB");
+
+template <bool SYM>
+__global__ void __launch_bounds__(BWDP_THREADS, 1)
+relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
+  using L = BwdPair64Smem;
+  constexpr int D = 64;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t bar0 = base + L::BARS;
+  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1);
+  auto FULL_T = [&](int s) { return BAR(2 + s); };
+  auto EMPTY_T = [&](int s) { return BAR(4 + s); };
+  auto FULL_S = [&](int s) { return BAR(6 + s); };
+  auto EMPTY_S = [&](int s) { return BAR(8 + s); };
+  const uint32_t S_FULL = BAR(10), S_EMPTY = BAR(11), G_FULL = BAR(12), G_EMPTY = BAR(13);
+  auto P_FULL = [&](int b) { return BAR(14 + b); };
+  auto P_EMPTY = [&](int b) { return BAR(16 + b); };
+  const uint32_t DXI_FULL = BAR(18), DXI_EMPTY = BAR(19), DRAIN_L = BAR(20), DRAIN_G = BAR(21);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
+
+  WaitCtl wc{p.status, abort_flag, p.timeout_ns};
+  constexpr uint32_t T_S = 0, T_DX0 = 256, T_P = 384;
+
+  if (threadIdx.x == 0) {
+    mbar_init(FULL_I, 1);
+    mbar_init(EMPTY_I, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(FULL_T(s), 1);
+      mbar_init(EMPTY_T(s), 1);
+      mbar_init(FULL_S(s), 1);
+      mbar_init(EMPTY_S(s), 1);
+      mbar_init(P_FULL(s), 1);
+      mbar_init(P_EMPTY(s), 4);
+    }
+    mbar_init(S_FULL, 1);
+    mbar_init(S_EMPTY, 16);
+    mbar_init(G_FULL, 16);
+    mbar_init(G_EMPTY, 1);
+    mbar_init(DXI_FULL, 1);
+    mbar_init(DXI_EMPTY, 4);
+    mbar_init(DRAIN_L, 1);
+    mbar_init(DRAIN_G, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == BWDP_LOGIT_WARP) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == BWD_TMA_WARP) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      for (int s = 0; s < p.n_seg; ++s) {
+        tma_prefetch_desc(&p.seg[s].tm_t);
+        tma_prefetch_desc(&p.seg[s].tm_s);
+        tma_prefetch_desc(&p.seg[s].tm_dx);
+      }
+      uint32_t nseq = 0, nJ = 0;
+      uint32_t armsT[2] = {0, 0}, armsS[2] = {0, 0};
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        int u, m;
+        decode_item(p, item, u, m);
+        const Unit U = decode_unit(p, u);
+        for (int w = 0; ok && w < 2; ++w) {
+          const int R0 = pair_seq_block(U, m, w);
+          if (R0 < 0) break;
+          const bool has1 = R0 + 1 < U.nblk;
+          if (!(ok = mbar_wait(EMPTY_I, (nseq & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
+          mbar_arrive_expect_tx(FULL_I, (has1 ? 4 : 2) * L::TILE);
+          tma_load_4d(base + L::XT_R0, &U.seg->tm_t, FULL_I, 0, U.tok0 + R0 * BM, U.h, U.b);
+          tma_load_4d(base + L::XS_R0, &U.seg->tm_s, FULL_I, 0, U.tok0 + R0 * BM, U.h, U.b);
+          if (has1) {
+            tma_load_4d(base + L::XT_R1, &U.seg->tm_t, FULL_I, 0, U.tok0 + (R0 + 1) * BM, U.h, U.b);
+            tma_load_4d(base + L::XS_R1, &U.seg->tm_s, FULL_I, 0, U.tok0 + (R0 + 1) * BM, U.h, U.b);
+          }
+          ++nseq;
+          const int nT = n_col_tiles_s<SYM>(p, U, has1 ? R0 + 1 : R0);
+          for (int J = 0; J < nT; ++J) {
+            const int st = nJ & 1;
+            if (!(ok = mbar_wait(EMPTY_T(st), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_T(st), L::TILE);
+            tma_load_4d(base + L::XT_J + st * L::TILE, &U.seg->tm_t, FULL_T(st), 0,
+                        U.tok0 + J * BN, U.h, U.b);
+            ++armsT[st];
+            if (!(ok = mbar_wait(EMPTY_S(st), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
+            mbar_arrive_expect_tx(FULL_S(st), L::TILE);
+            tma_load_4d(base + L::XS_J + st * L::TILE, &U.seg->tm_s, FULL_S(st), 0,
+                        U.tok0 + J * BN, U.h, U.b);
+            ++armsS[st];
+            ++nJ;
+          }
+        }
+      }
+      if (nseq) mbar_wait_drain(FULL_I, (nseq - 1) & 1, kDrainNs);
+      for (int s = 0; s < 2; ++s) {
+        if (armsT[s]) mbar_wait_drain(FULL_T(s), (armsT[s] - 1) & 1, kDrainNs);
+        if (armsS[s]) mbar_wait_drain(FULL_S(s), (armsS[s] - 1) & 1, kDrainNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == BWDP_LOGIT_WARP || warp == BWDP_GRAD_WARP) {
+    // ------------------------------------------------------------ MMA
+    // One warp issues the logit MMAs of the next tile as soon as the row
+    // warps have read the current one; the other the gradient MMAs of the
+    // tile whose G was just stored.  Each runs its loop converged; one
+    // elected lane issues.
+    const bool is_logit = warp == BWDP_LOGIT_WARP;
+    const uint32_t lead = elect_leader();
+    constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);
+    constexpr uint32_t IDESC_GX = idesc_bf16_f32(BM, D, 0, 1);   // A = G (K-major), B = X_s[J] (MN)
+    constexpr uint32_t IDESC_P = idesc_bf16_f32(BM, D, 1, 1);    // A = G^T (MN), B = X_s[R] (MN)
+    const uint32_t HI_1024 = sw128_desc_hi(1024);
+    const uint32_t dXtR_k[2] = {sw128_desc_lo(base + L::XT_R0, 16), sw128_desc_lo(base + L::XT_R1, 16)};
+    const uint32_t dXsR_k[2] = {sw128_desc_lo(base + L::XS_R0, 16), sw128_desc_lo(base + L::XS_R1, 16)};
+    const uint32_t dXsR_mn[2] = {sw128_desc_lo(base + L::XS_R0, L::TILE),
+                                 sw128_desc_lo(base + L::XS_R1, L::TILE)};
+    const uint32_t dXtJ_k0 = sw128_desc_lo(base + L::XT_J, 16);
+    const uint32_t dXsJ_k0 = sw128_desc_lo(base + L::XS_J, 16);
+    const uint32_t dXsJ_mn0 = sw128_desc_lo(base + L::XS_J, L::TILE);
+    const uint32_t dG_k = sw128_desc_lo(base + L::G, 16);
+    const uint32_t dG_mn = sw128_desc_lo(base + L::G, L::TILE);
+    constexpr uint32_t J_STEP = L::TILE >> 4, BOX_STEP = L::TILE >> 4;
+    uint32_t nseq = 0, nJ = 0, nt = 0, np = 0;
+    bool ok = true, issued = false;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      int u, m;
+      decode_item(p, item, u, m);
+      const Unit U = decode_unit(p, u);
+      for (int w = 0; ok && w < 2; ++w) {
+        const int R0 = pair_seq_block(U, m, w);
+        if (R0 < 0) break;
+        const bool has1 = R0 + 1 < U.nblk;
+        const int nT0 = n_col_tiles_s<SYM>(p, U, R0);
+        const int nT = has1 ? n_col_tiles_s<SYM>(p, U, R0 + 1) : nT0;
+        if (!(ok = mbar_wait_warp(FULL_I, nseq & 1, wc, W_MMA_FULL_I))) break;
+        bool first_seq = true;
+        for (int J = 0; ok && J < nT; ++J) {
+          const int st = nJ & 1;
+          for (int rs = 0; rs < 2; ++rs) {
+            if (rs == 0 && J >= nT0) continue;
+            if (rs == 1 && !has1) continue;
+            const bool first_p = rs == 0 || J >= nT0;
+            const bool last_p = rs == 1 || !has1;
+            if (is_logit) {
+              // Z_t, Z_s of tile (R, J): M = 128 rows, N = 128 columns, K = 64
+              if (!(ok = mbar_wait_warp(FULL_T(st), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+              if (!(ok = mbar_wait_warp(S_EMPTY, (nt & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
+              tc_fence_after();
+              const uint32_t xtj = dXtJ_k0 + st * J_STEP, xsj = dXsJ_k0 + st * J_STEP;
+#pragma unroll
+              for (int k = 0; k < D / 16; ++k)
+                umma_bf16_w_lead(lead, tmem + T_S, dXtR_k[rs] + k * 2, HI_1024, xtj + k * 2,
+                                 HI_1024, IDESC_S, k > 0 ? 1u : 0u);
+              issued = true;
+              if (last_p) umma_commit_lead(lead, EMPTY_T(st));
+              if (!(ok = mbar_wait_warp(FULL_S(st), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+              tc_fence_after();
+#pragma unroll
+              for (int k = 0; k < D / 16; ++k)
+                umma_bf16_w_lead(lead, tmem + T_S + BN, dXsR_k[rs] + k * 2, HI_1024, xsj + k * 2,
+                                 HI_1024, IDESC_S, k > 0 ? 1u : 0u);
+              umma_commit_lead(lead, S_FULL);
+            } else {
+              // dX_R += G X_s[J] and P (+)= G^T X_s[R] for tile (R, J).  G_FULL
+              // implies the tile's logits (hence its column tiles) are complete.
+              const int pb = np & 1;
+              if (!(ok = mbar_wait_warp(G_FULL, nt & 1, wc, W_MMA_G_FULL))) break;
+              if (first_p && !(ok = mbar_wait_warp(P_EMPTY(pb), ((np >> 1) & 1) ^ 1, wc, W_MMA_P_EMPTY)))
+                break;
+              if (first_seq && !(ok = mbar_wait_warp(DXI_EMPTY, (nseq & 1) ^ 1, wc, W_MMA_DXI_EMPTY)))
+                break;
+              first_seq = false;
+              tc_fence_after();
+              const uint32_t xsj = dXsJ_mn0 + st * J_STEP;
+              // M = i, N = c (64), K = j (128): G K-major steps 32 B in a row and a
+              // box every 4 steps; X_s[J] MN-major steps 16 rows (2 KB)
+#pragma unroll
+              for (int k = 0; k < BN / 16; ++k)
+                umma_bf16_w_lead(lead, tmem + T_DX0 + rs * D, dG_k + (k >> 2) * BOX_STEP + (k & 3) * 2,
+                                 HI_1024, xsj + k * 128, HI_1024, IDESC_GX, (J > 0 || k > 0) ? 1u : 0u);
+              // M = j (128, two 64-column boxes of G, LBO = box), N = c (64), K = i (128)
+#pragma unroll
+              for (int k = 0; k < BM / 16; ++k)
+                umma_bf16_w_lead(lead, tmem + T_P + pb * D, dG_mn + k * 128, HI_1024,
+                                 dXsR_mn[rs] + k * 128, HI_1024, IDESC_P,
+                                 (!first_p || k > 0) ? 1u : 0u);
+              issued = true;
+              umma_commit_lead(lead, G_EMPTY);
+              if (last_p) {
+                umma_commit_lead(lead, P_FULL(pb));
+                umma_commit_lead(lead, EMPTY_S(st));
+                ++np;
+              }
+            }
+            ++nt;
+          }
+          ++nJ;
+        }
+        if (!ok) break;
+        if (!is_logit) {
+          umma_commit_lead(lead, EMPTY_I);
+          umma_commit_lead(lead, DXI_FULL);
+        }
+        ++nseq;
+      }
+    }
+    if (issued) {
+      const uint32_t drain = is_logit ? DRAIN_L : DRAIN_G;
+      umma_commit_lead(lead, drain);
+      mbar_wait_drain(drain, 0, kDrainNs);
+    }
+    __syncwarp();
+  } else if (warp >= BWD_EPI_WARP) {
+    // ------------------------------------------------------- epilogue
+    // Every f32 addition into dX goes out as a TMA reduce-add of a 32 x 32
+    // box staged in this warp's 4 KB of shared memory (128-byte swizzle, one
+    // 128-byte row per lane).  Lane 32q + l of P holds dX[J*128 + 32q + l][0:64].
+    const int q = warp - BWD_EPI_WARP;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t stg = base + L::STG + q * L::STG_BYTES;
+    const uint32_t rowp = stg + lane * 128;
+    uint32_t np = 0, nseq = 0;
+    bool ok = true;
+    // stage 32 columns of this lane's row and add the box at (c0, row0)
+    auto stage_add = [&](const float (&v)[32], const CUtensorMap* map, int c0, int row0, const Unit& U) {
+      if (lane == 0) bulk_wait_read<0>();   // the previous box has left the buffer
+      __syncwarp();
+#pragma unroll
+      for (int k4 = 0; k4 < 8; ++k4)
+        st_shared_v4(rowp + ((k4 ^ (lane & 7)) << 4), __float_as_uint(v[4 * k4]),
+                     __float_as_uint(v[4 * k4 + 1]), __float_as_uint(v[4 * k4 + 2]),
+                     __float_as_uint(v[4 * k4 + 3]));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (row0 < p.N) tma_reduce_add_4d(map, stg, c0, row0, U.h, U.b);
+        bulk_commit();
+      }
+    };
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      int u, m;
+      decode_item(p, item, u, m);
+      const Unit U = decode_unit(p, u);
+      for (int w = 0; ok && w < 2; ++w) {
+        const int R0 = pair_seq_block(U, m, w);
+        if (R0 < 0) break;
+        const bool has1 = R0 + 1 < U.nblk;
+        const int nT = n_col_tiles_s<SYM>(p, U, has1 ? R0 + 1 : R0);
+        for (int J = 0; J < nT; ++J) {
+          const int b = np & 1;
+          ok = mbar_wait(P_FULL(b), (np >> 1) & 1, wc, W_EPI_P_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int cb = 0; cb < D / 32; ++cb) {
+            float v[32];
+            tmem_ld32(tmem + lane_addr + T_P + b * D + cb * 32, v);
+            tmem_wait_ld();
+            if (cb == D / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(P_EMPTY(b));
+            }
+            stage_add(v, &U.seg->tm_dx, cb * 32, U.tok0 + J * BN + q * 32, U);
+          }
+          ++np;
+        }
+        if (!ok) break;
+        // dX rows of the pair: lane = row, 32-column boxes
+        ok = mbar_wait(DXI_FULL, nseq & 1, wc, W_EPI_DXI_FULL);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        for (int rs = 0; rs < 2; ++rs) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tmem_ld32(tmem + lane_addr + T_DX0 + rs * D + c * 32, v);
+            tmem_wait_ld();
+            if (rs == 1 && c == D / 32 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(DXI_EMPTY);
+            }
+            if (rs == 1 && !has1) continue;
+            stage_add(v, &U.seg->tm_dx, c * 32, U.tok0 + (R0 + rs) * BM + q * 32, U);
+          }
+        }
+        ++nseq;
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  } else {
+    // --------------------------------------------------- row warpgroups
+    const int q = warp & 3;
+    const int wg = warp >> 2;      // 32-column quarter of each 128-column tile
+    const int r = q * 32 + lane;
+    const float sl2 = p.sl2;
+    // this thread's 64-byte slice of row r of G: box wg/2, chunks 4*(wg&1)..+3
+    const uint32_t gsm = base + L::G + (wg >> 1) * L::TILE + r * 128;
+    uint32_t nt = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+      int u, m;
+      decode_item(p, item, u, m);
+      const Unit U = decode_unit(p, u);
+      for (int w = 0; ok && w < 2; ++w) {
+        const int R0 = pair_seq_block(U, m, w);
+        if (R0 < 0) break;
+        const bool has1 = R0 + 1 < U.nblk;
+        const int nT0 = n_col_tiles_s<SYM>(p, U, R0);
+        const int nT = has1 ? n_col_tiles_s<SYM>(p, U, R0 + 1) : nT0;
+        const int Lu = U.len;
+        // per-row constants of both row blocks
+        float bt[2], bs[2], mul[2];
+        int lim[2];
+#pragma unroll
+        for (int rs = 0; rs < 2; ++rs) {
+          const int row = (R0 + rs) * BM + r;
+          const bool rvalid = row < Lu && (rs == 0 || has1);
+          bt[rs] = bs[rs] = mul[rs] = 0.f;
+          if (rvalid) {
+            const float4 st4 = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + row];
+            bt[rs] = -st4.y * kLog2e;
+            bs[rs] = -st4.z * kLog2e;
+            const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(Lu);
+            mul[rs] = up * p.scale;   // the logit scale of dX_s is folded into G
+          }
+          lim[rs] = !rvalid ? -1 : (p.causal ? min(row, Lu - 1) : Lu - 1);
+        }
+        const float2 sl2v = make_float2(sl2, sl2), m1 = make_float2(-1.f, -1.f);
+        for (int J = 0; ok && J < nT; ++J) {
+          for (int rs = 0; rs < 2; ++rs) {
+            if (rs == 0 && J >= nT0) continue;
+            if (rs == 1 && !has1) continue;
+            ok = mbar_wait(S_FULL, nt & 1, wc, W_SM_S_FULL);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + T_S + wg * 32;
+            const float btr = rs ? bt[1] : bt[0], bsr = rs ? bs[1] : bs[0];
+            const float mr = rs ? mul[1] : mul[0];
+            const int limr = rs ? lim[1] : lim[0];
+            const int col0 = J * BN + wg * 32;
+            if constexpr (SYM) {
+              // full mask: 4 exps per entry off the diagonal tile, so the exps
+              // bound this mode; the logits are read in two 16-column halves
+              // (the second half releases the buffer) to keep registers free
+              // for the partners' statistics
+              const bool off = J < R0 + rs;
+#pragma unroll 1
+              for (int hf = 0; hf < 2; ++hf) {
+                float t[16], s[16];
+                tmem_ld16(ta + hf * 16, t);
+                tmem_ld16(ta + BN + hf * 16, s);
+                tmem_wait_ld();
+                if (hf == 1) {
+                  tc_fence_before();
+                  __syncwarp();
+                  if (lane == 0) mbar_arrive(S_EMPTY);
+                } else {
+                  ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
+                  ok = __all_sync(0xffffffffu, ok);
+                  if (!ok) break;
+                }
+                form_g_store<16>(t, s, btr, bsr, mr, col0 + hf * 16, limr, off, U, p, gsm,
+                                 (wg & 1) * 4 + hf * 2, r);
+              }
+              if (!ok) break;
+            } else {
+            float t[32], s[32];
+            tmem_ld32(ta, t);
+            tmem_ld32(ta + BN, s);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(S_EMPTY);
+            const float2 btv = make_float2(btr, btr), bsv = make_float2(bsr, bsr),
+                         mulv = make_float2(mr, mr);
+            const bool need_mask = col0 + 31 > limr;
+            // the previous tile's gradient MMAs have read G (they were issued
+            // a whole exp pass ago): wait first, then store each 16-byte chunk
+            // as soon as it is formed, which keeps few values live at once
+            ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int k2 = 0; k2 < 8; k2 += 2) {
+                const int k = q4 * 8 + k2;
+                const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
+                const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
+                const float2 et = ex2_approx2(at), es = ex2_approx2(as);
+                float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
+                if (need_mask) {
+                  g.x = (col0 + k <= limr) ? g.x : 0.f;
+                  g.y = (col0 + k + 1 <= limr) ? g.y : 0.f;
+                }
+                pk[k2 >> 1] = pack_bf16x2(g.x, g.y);
+              }
+              const int cc = (wg & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
+              st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+            }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -1789,8 +2360,25 @@ cudaError_t tc_launch_fwd(const TcParams& p, int d, int grid, cudaStream_t strea
 // item of the kernel chosen, whichever is fewer.
 cudaError_t tc_launch_bwd(const TcParams& p, int d, int max_grid, cudaStream_t stream) {
   int grid = p.n_items < max_grid ? p.n_items : max_grid;
-  if (d == 64) return grid ? launch_bwd<64>(p, grid, stream) : cudaSuccess;
-  if (p.nblk <= kPairMinBlocks - 1) {
+  if (d == 64) {
+    // work items of the paired-block kernel: ceil(npb / 2) per unit
+    TcParams q = p;
+    q.n_pairs = ((p.nblk + 1) / 2 + 1) / 2;
+    q.n_local = q.part < q.n_pairs ? (q.n_pairs - q.part + q.n_parts - 1) / q.n_parts : 0;
+    q.n_items = q.n_units * q.n_local;
+    if (q.n_items == 0) return cudaSuccess;
+    grid = q.n_items < max_grid ? q.n_items : max_grid;
+    auto k = p.causal ? relkl_bwd_pair64_kernel<false> : relkl_bwd_pair64_kernel<true>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         BwdPair64Smem::ALLOC);
+    if (e != cudaSuccess) return e;
+    k<<<grid, BWDP_THREADS, BwdPair64Smem::ALLOC, stream>>>(q);
+    return cudaGetLastError();
+  }
+  // full masks take the paired-block kernel at every N (it serves both
+  // orientations of each off-diagonal tile); causal ones with few row blocks
+  // the one-block kernel, whose finer work items balance better
+  if (p.causal && p.nblk <= kPairMinBlocks - 1) {
     if (!grid) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(relkl_bwd_tc64_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1806,11 +2394,11 @@ cudaError_t tc_launch_bwd(const TcParams& p, int d, int max_grid, cudaStream_t s
   q.n_items = q.n_units * q.n_local;
   if (q.n_items == 0) return cudaSuccess;
   grid = q.n_items < max_grid ? q.n_items : max_grid;
-  cudaError_t e = cudaFuncSetAttribute(relkl_bwd_pair_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto k = p.causal ? relkl_bwd_pair_kernel<false> : relkl_bwd_pair_kernel<true>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        BwdPairSmem::ALLOC);
   if (e != cudaSuccess) return e;
-  relkl_bwd_pair_kernel<<<grid, BWDP_THREADS, BwdPairSmem::ALLOC, stream>>>(q);
+  k<<<grid, BWDP_THREADS, BwdPairSmem::ALLOC, stream>>>(q);
   return cudaGetLastError();
 }
 

@@ -369,7 +369,7 @@ def relkl_rope_bwd(dx_post: torch.Tensor, base: float, pos_scale: float = 1.0,
 
 
 def relkl_weight_grad(h: torch.Tensor, dx_pre: torch.Tensor, *, out: Optional[torch.Tensor] = None,
-                      stream=None) -> torch.Tensor:
+                      ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """dW [D, cols] fp32 = h^T dx_pre over token rows (h [..., D], dx_pre [..., cols], bf16)."""
     _cuda(h, "h")
     _cuda(dx_pre, "dx_pre")
@@ -387,9 +387,10 @@ def relkl_weight_grad(h: torch.Tensor, dx_pre: torch.Tensor, *, out: Optional[to
     if out is None:
         out = torch.empty(D, cols, dtype=torch.float32, device=h.device)
     _check_out(out, (D, cols), "dw", h.device)
+    ws = workspace(h.device) if ws is None else ws
     with torch.cuda.device(h.device):
         code = _abi.lib().relkl_weight_grad(rows, D, cols, _ptr(h), _ptr(dx_pre), _ptr(out),
-                                            _stream(h.device, stream))
+                                            _ptr(ws), ws.numel(), _stream(h.device, stream))
     check(code, "relkl_weight_grad")
     return out
 

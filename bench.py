@@ -63,9 +63,12 @@ def bwd_kernel_name(w) -> str:
     if w.dtype != "bf16" or w.d not in (64, 128):
         return "relkl_bwd_simt_kernel"
     if w.d == 64:
-        return "relkl_bwd_tc_kernel"
-    # 128-row blocks: more than 32 of them take the kernel that pairs adjacent blocks
-    return "relkl_bwd_pair_kernel" if (w.N + 127) // 128 > 32 else "relkl_bwd_tc64_kernel"
+        return "relkl_bwd_pair64_kernel"
+    # full masks, and causal ones with more than 32 row blocks, take the kernel
+    # that pairs adjacent row blocks
+    if not w.causal or (w.N + 127) // 128 > 32:
+        return "relkl_bwd_pair_kernel"
+    return "relkl_bwd_tc64_kernel"
 
 
 def traffic_record(kernel: str):

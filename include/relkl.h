@@ -272,18 +272,18 @@ relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const fl
  *
  *   dw[D, cols] = h[rows, D]^T dx_pre[rows, cols]
  *
- * (rows = B*N tokens, cols = heads * d), overwriting dw.  One dense GEMM on
- * the tensor cores through cuBLAS: bf16 operands, float32 accumulation and
- * result.  The library keeps one cuBLAS handle per device, created on the
- * first call without a workspace; calls are serialised on it.
+ * (rows = B*N tokens, cols = heads * d), overwriting dw: one dense GEMM on
+ * the tensor cores (the library's own tcgen05 kernel), bf16 operands, float32
+ * accumulation and result.
  *   h      : bf16 [rows, D] row-major (the student's hidden states), in.
  *   dx_pre : bf16 [rows, cols] row-major (relkl_rope_bwd's output), in.
  *   dw     : float [D, cols] row-major, out.
+ *   ws     : the workspace record of the other calls (bounded waits).
  * 1 <= rows <= 2^31 - 1, D >= 1, cols >= 1; pointers 16-byte aligned and
- * D, cols multiples of 8.  RELKL_ERR_INVALID otherwise; RELKL_ERR_CUDA with
- * the cuBLAS status in relkl_last_cuda_error() when cuBLAS fails.            */
+ * D, cols multiples of 8.  RELKL_ERR_INVALID otherwise.                      */
 relkl_status relkl_weight_grad(int64_t rows, int32_t D, int32_t cols, const void* h,
-                               const void* dx_pre, float* dw, void* stream);
+                               const void* dx_pre, float* dw, void* ws, size_t ws_bytes,
+                               void* stream);
 
 #ifdef __cplusplus
 }

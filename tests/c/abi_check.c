@@ -48,7 +48,8 @@ int main(void) {
         "rope_bwd with odd d");
   CHECK(relkl_rope_bwd(0, 2, 8, 64, NULL, &rope, RELKL_BF16, NULL, NULL) == RELKL_OK,
         "rope_bwd with no tokens is a no-op");
-  CHECK(relkl_weight_grad(0, 64, 64, f, f, f, NULL) == RELKL_ERR_INVALID, "weight_grad rows=0");
+  CHECK(relkl_weight_grad(0, 64, 64, f, f, f, f, 256, NULL) == RELKL_ERR_INVALID,
+        "weight_grad rows=0");
 
   uint64_t old = relkl_set_wait_timeout_ns(123456789ull);
   CHECK(relkl_set_wait_timeout_ns(old) == 123456789ull, "timeout round trip");

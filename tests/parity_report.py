@@ -99,7 +99,7 @@ def run_chain(out):
     for r in "qkv":
         g, w = to_np(got[r]), ref[r]
         rel = float(np.abs(g - w).max() / np.abs(w).max())
-        out.append((f"chain_small dW_{r} [{w.shape[0]}x{w.shape[1]}]", "RoPE bwd + cuBLAS GEMM",
+        out.append((f"chain_small dW_{r} [{w.shape[0]}x{w.shape[1]}]", "RoPE bwd + tcgen05 GEMM",
                     "every weight", float("nan"), float("nan"), rel, rel / DX_TOL_BF16))
 
 

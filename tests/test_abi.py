@@ -161,7 +161,9 @@ def test_weight_grad_validation():
         (8, 64, 12, p, p, p), (2 ** 31, 64, 64, p, p, p), (8, 64, 64, None, p, p),
         (8, 64, 64, p, None, p), (8, 64, 64, p, p, None), (8, 64, 64, ctypes.c_void_p(4104), p, p),
     ]:
-        assert lib.relkl_weight_grad(rows, D, cols, h, dx, dw, None) == inv
+        assert lib.relkl_weight_grad(rows, D, cols, h, dx, dw, p, 256, None) == inv
+    # a missing workspace is refused after the shapes are accepted
+    assert lib.relkl_weight_grad(8, 64, 64, p, p, p, None, 0, None) == _abi.RELKL_ERR_WORKSPACE
 
 
 def test_binding_rejects_bad_outputs_before_the_call():

@@ -147,6 +147,16 @@ def test_simt_bf16_unsupported_head_dim():
     check_full(xt, xs, dx_tol=FP32, path=2)
 
 
+@pytest.mark.parametrize("N,d", [(700, 128), (4480, 128), (513, 64), (4300, 64)])
+def test_full_mask_upstream_gradient(N, d):
+    """Full masks run the symmetric schedule: each off-diagonal tile also forms
+    the transposed entry's gradient from the column row's statistics and
+    upstream gradient, so a row-dependent dkl must reach both orientations."""
+    xt, xs = q_inputs(1, 1, N, d, seed=N + 3 * d, causal=False)
+    dkl = torch.randn(1, 1, N, generator=torch.Generator().manual_seed(N)) / N
+    check_full(xt, xs, causal=False, dkl=dkl, path=1)
+
+
 def test_upstream_gradient():
     xt, xs = q_inputs(2, 2, 260, 128, seed=11)
     dkl = torch.randn(2, 2, 260, generator=torch.Generator().manual_seed(2)) / 260
@@ -339,6 +349,13 @@ def test_config_d64_h32_n32k():
     # sampled rows of one unit of each relation
     w = workload.CONFIGS["d64_h32_n32k"]
     units = [("q", 0, 0), ("k", 0, 17), ("v", 0, 31)]
+    _sampled(w, units, dx_units=set(units))
+
+
+def test_config_full_h32_n16k():
+    # full mask at 16K (the symmetric paired-block backward)
+    w = workload.CONFIGS["full_h32_n16k"]
+    units = [("q", 0, 5), ("k", 0, 17), ("v", 0, 31)]
     _sampled(w, units, dx_units=set(units))
 
 

@@ -84,5 +84,9 @@ def test_bench_names_the_backward_kernel_the_library_launches():
         w = workload.tiny_custom(N=N, d=128, dtype="bf16")
         want = "relkl_bwd_pair_kernel" if (N + 127) // 128 >= min_blocks else "relkl_bwd_tc64_kernel"
         assert bench.bwd_kernel_name(w) == want, N
-    assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=64, dtype="bf16")) == "relkl_bwd_tc_kernel"
+    # full masks take the paired-block kernel at every N (the symmetric schedule)
+    assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=128, dtype="bf16", causal=False)) \
+        == "relkl_bwd_pair_kernel"
+    assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=64, dtype="bf16")) == \
+        "relkl_bwd_pair64_kernel"
     assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=64, dtype="fp32")) == "relkl_bwd_simt_kernel"

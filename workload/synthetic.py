@@ -94,6 +94,11 @@ CONFIGS: Dict[str, Workload] = {
     "d64_h32_n32k": Workload("d64_h32_n32k", B=1, H=32, H_kv=32, N=32768, d=64,
                              dtype="bf16", causal=True, relations=("q", "k", "v"),
                              rope_base=1e4, pi_factor=8.0, v_noise=0.1, seed=6),
+    # full (non-causal) mask: every row sees every token (the pages leave the
+    # mask M open; this is the unmasked reading), 16K tokens
+    "full_h32_n16k": Workload("full_h32_n16k", B=1, H=32, H_kv=32, N=16384, d=128,
+                              dtype="bf16", causal=False, relations=("q", "k", "v"),
+                              rope_base=1e4, pi_factor=8.0, v_noise=0.1, seed=7),
 }
 
 SWEEP_N = (1024, 2048, 4096, 8192, 16384, 32768, 65536)
