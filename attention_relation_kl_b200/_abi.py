@@ -21,7 +21,7 @@ EXPORTS = ("relkl_workspace_bytes", "relkl_workspace_init", "relkl_fwd", "relkl_
            "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_get_device_error",
            "relkl_set_wait_timeout_ns", "relkl_status_string", "relkl_last_cuda_error",
            "relkl_path_for", "relkl_fwd_noalloc", "relkl_rope_bwd", "relkl_weight_grad",
-           "relkl_fwd_qkv_part", "relkl_bwd_qkv_part")
+           "relkl_fwd_qkv_part", "relkl_bwd_qkv_part", "relkl_check_schedule")
 
 
 class relkl_desc(ctypes.Structure):
@@ -69,6 +69,9 @@ def _declare(lib):
     lib.relkl_bwd_qkv_part.argtypes = [ctypes.c_int32, ctypes.POINTER(relkl_desc), _PV, _PV, _PV,
                                        _PV, _PV, ctypes.c_int32, ctypes.c_int32, _vp,
                                        ctypes.c_size_t, _vp]
+    lib.relkl_check_schedule.restype = ctypes.c_int
+    lib.relkl_check_schedule.argtypes = [ctypes.c_int32, ctypes.POINTER(relkl_desc), ctypes.c_int32,
+                                         ctypes.c_int32, _PV, _PV, ctypes.c_char_p, ctypes.c_size_t]
     lib.relkl_get_device_error.restype = ctypes.c_int
     lib.relkl_get_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.relkl_set_wait_timeout_ns.restype = ctypes.c_uint64

@@ -44,12 +44,18 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile librelkl.so if any source is newer; returns its path."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, checks: bool = False) -> str:
+    """Compile librelkl.so if any source is newer; returns its path.
+
+    ``checks`` (or RELKL_CHECKS=1 in the environment) builds the debug variant
+    that replays every tensor-core launch's schedule on the host first
+    (relkl_check_schedule) and refuses a launch whose schedule is unsound."""
+    checks = checks or os.environ.get("RELKL_CHECKS") == "1"
+    if not force and not checks and not _stale():
         return LIB
     tmp = LIB + ".tmp"
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
+    cmd = [nvcc_path(), *NVCC_FLAGS, *(["-DRELKL_CHECKS"] if checks else []),
+           "-I", os.path.join(ROOT, "include"),
            *[os.path.join(CSRC, f) for f in SOURCES], "-ldl", "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
@@ -61,4 +67,4 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, checks="--checks" in sys.argv))

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -22,6 +23,8 @@ cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t strea
 cudaError_t simt_launch_fwd(const SimtParams& p, cudaStream_t stream);
 cudaError_t simt_launch_bwd(const SimtParams& p, cudaStream_t stream);
 cudaError_t launch_zero(float* ptr, int64_t n, int num_sms, cudaStream_t stream);
+int schedule_check(const TcParams& p0, int d, bool bwd, int n_parts, const int* const* lens,
+                   const int* const* offs, char* why, size_t why_len);
 cudaError_t launch_rope_bwd(const float* dx, void* out, int B, int H, int N, int d, bool bf16_out,
                             double base, double pos_scale, double pos_offset, int apply,
                             cudaStream_t stream);
@@ -232,18 +235,15 @@ bool use_tc(int32_t n_rel, const relkl_desc* descs, const void* const* xt, const
   return true;
 }
 
-relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const* xt,
-                      const void* const* xs, TcParams* p, void* ws, int part = 0,
-                      int n_parts = 1) {
+// The schedule fields of a tensor-core launch (everything but the tensor
+// maps and pointers): shared by the launch and the host schedule check.
+void fill_schedule(int32_t n_rel, const relkl_desc* descs, TcParams* p, int part, int n_parts) {
   std::memset(p, 0, sizeof(*p));
   const relkl_desc& d0 = descs[0];
   int seg = 0, ub = 0;
   for (int r = 0; r < n_rel; ++r) {
     if (n_units(descs[r]) == 0) continue;
     TcSeg& s = p->seg[seg];
-    relkl_status st = encode_x(&s.tm_t, descs[r], xt[r]);
-    if (st != RELKL_OK) return st;
-    if ((st = encode_x(&s.tm_s, descs[r], xs[r])) != RELKL_OK) return st;
     s.B = descs[r].cu_seqlens ? descs[r].n_seq : descs[r].B;
     s.H = descs[r].H;
     s.lengths = descs[r].lengths;
@@ -267,6 +267,19 @@ relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const*
   p->causal = d0.causal;
   p->scale = logit_scale(d0);
   p->sl2 = p->scale * 1.4426950408889634f;
+}
+
+relkl_status build_tc(int32_t n_rel, const relkl_desc* descs, const void* const* xt,
+                      const void* const* xs, TcParams* p, void* ws, int part = 0,
+                      int n_parts = 1) {
+  fill_schedule(n_rel, descs, p, part, n_parts);
+  for (int r = 0, seg = 0; r < n_rel; ++r) {
+    if (n_units(descs[r]) == 0) continue;
+    TcSeg& s = p->seg[seg++];
+    relkl_status st = encode_x(&s.tm_t, descs[r], xt[r]);
+    if (st != RELKL_OK) return st;
+    if ((st = encode_x(&s.tm_s, descs[r], xs[r])) != RELKL_OK) return st;
+  }
   p->status = reinterpret_cast<DevStatus*>(ws);
   p->timeout_ns = g_timeout_ns.load();
   return RELKL_OK;
@@ -347,6 +360,36 @@ int32_t relkl_path_for(const relkl_desc* desc) {
 
 namespace {
 
+#ifdef RELKL_CHECKS
+// Debug builds (-DRELKL_CHECKS): replay the launch's schedule on the host
+// before enqueueing it (synchronous copies of lengths / packed offsets).
+relkl_status debug_schedule_check(int32_t n_rel, const relkl_desc* descs, bool bwd, int part,
+                                  int n_parts) {
+  std::vector<std::vector<int32_t>> lens(n_rel), offs(n_rel);
+  const int32_t* lp[kMaxSeg] = {nullptr, nullptr, nullptr};
+  const int32_t* op[kMaxSeg] = {nullptr, nullptr, nullptr};
+  for (int r = 0; r < n_rel; ++r) {
+    if (descs[r].lengths) {
+      lens[r].resize(descs[r].B);
+      if (cudaMemcpy(lens[r].data(), descs[r].lengths, 4 * descs[r].B, cudaMemcpyDeviceToHost) !=
+          cudaSuccess)
+        return RELKL_ERR_CUDA;
+      lp[r] = lens[r].data();
+    }
+    if (descs[r].cu_seqlens) {
+      offs[r].resize(descs[r].n_seq + 1);
+      if (cudaMemcpy(offs[r].data(), descs[r].cu_seqlens, 4 * (descs[r].n_seq + 1),
+                     cudaMemcpyDeviceToHost) != cudaSuccess)
+        return RELKL_ERR_CUDA;
+      op[r] = offs[r].data();
+    }
+  }
+  (void)part;
+  char why[256];
+  return relkl_check_schedule(n_rel, descs, bwd ? 1 : 0, n_parts, lp, op, why, sizeof why);
+}
+#endif
+
 relkl_status fwd_impl(int32_t n_rel, const relkl_desc* descs, const void* const* x_t,
                       const void* const* x_s, float* const* kl, float* const* stats, int32_t part,
                       int32_t n_parts, void* ws, size_t ws_bytes, void* stream) {
@@ -365,6 +408,9 @@ relkl_status fwd_impl(int32_t n_rel, const relkl_desc* descs, const void* const*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (use_tc(n_rel, descs, x_t, x_s)) {
+#ifdef RELKL_CHECKS
+    if ((s = debug_schedule_check(n_rel, descs, false, part, n_parts)) != RELKL_OK) return s;
+#endif
     TcParams p;
     if ((s = build_tc(n_rel, descs, x_t, x_s, &p, ws, part, n_parts)) != RELKL_OK) return s;
     set_seg_outputs(&p, n_rel, descs, kl, stats, nullptr, nullptr, nullptr);
@@ -405,6 +451,9 @@ relkl_status bwd_impl(int32_t n_rel, const relkl_desc* descs, const void* const*
   TcParams tp;
   SimtParams sp;
   if (tc) {
+#ifdef RELKL_CHECKS
+    if ((s = debug_schedule_check(n_rel, descs, true, part, n_parts)) != RELKL_OK) return s;
+#endif
     if ((s = build_tc(n_rel, descs, x_t, x_s, &tp, ws, part, n_parts)) != RELKL_OK) return s;
     set_seg_outputs(&tp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);
     for (int r = 0, seg = 0; r < n_rel; ++r) {
@@ -520,6 +569,43 @@ const char* relkl_status_string(relkl_status s) {
 }
 
 int32_t relkl_last_cuda_error(void) { return g_last_cuda; }
+
+relkl_status relkl_check_schedule(int32_t n_rel, const relkl_desc* descs, int32_t is_bwd,
+                                  int32_t n_parts, const int32_t* const* host_lengths,
+                                  const int32_t* const* host_cu_seqlens, char* why,
+                                  size_t why_len) {
+  if (why && why_len) why[0] = 0;
+  if (n_rel < 1 || n_rel > kMaxSeg || !descs || n_parts < 1) return RELKL_ERR_INVALID;
+  int64_t units = 0;
+  for (int r = 0; r < n_rel; ++r) {
+    relkl_status s = check_desc(&descs[r]);
+    if (s != RELKL_OK) return s;
+    if (descs[r].N != descs[0].N || descs[r].causal != descs[0].causal ||
+        (descs[r].cu_seqlens == nullptr) != (descs[0].cu_seqlens == nullptr) ||
+        descs[r].max_seqlen != descs[0].max_seqlen || descs[r].d != descs[0].d)
+      return RELKL_ERR_INVALID;
+    if ((descs[r].lengths && (!host_lengths || !host_lengths[r])) ||
+        (descs[r].cu_seqlens && (!host_cu_seqlens || !host_cu_seqlens[r])))
+      return RELKL_ERR_INVALID;
+    units += n_units(descs[r]);
+  }
+  if (!tc_shape(descs[0])) return RELKL_ERR_UNSUPPORTED;
+  if (units == 0 || descs[0].N == 0) return RELKL_OK;
+  TcParams p;
+  fill_schedule(n_rel, descs, &p, 0, 1);
+  // host copies in the launch's segment order (relations without units have none)
+  const int* lens[kMaxSeg] = {nullptr, nullptr, nullptr};
+  const int* offs[kMaxSeg] = {nullptr, nullptr, nullptr};
+  for (int r = 0, seg = 0; r < n_rel; ++r) {
+    if (n_units(descs[r]) == 0) continue;
+    lens[seg] = host_lengths ? host_lengths[r] : nullptr;
+    offs[seg] = host_cu_seqlens ? host_cu_seqlens[r] : nullptr;
+    ++seg;
+  }
+  return schedule_check(p, descs[0].d, is_bwd != 0, n_parts, lens, offs, why, why_len) == 0
+             ? RELKL_OK
+             : RELKL_ERR_INVALID;
+}
 
 relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const float* dx_post,
                             const relkl_rope* rope, int32_t out_dtype, void* dx_pre,

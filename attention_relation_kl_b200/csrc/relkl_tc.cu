@@ -36,6 +36,8 @@
 // loop, waits for its own copies and MMAs in flight and the CTA frees its TMEM
 // and exits.
 #include <cstdint>
+#include <cstdio>
+#include <vector>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -61,12 +63,18 @@ struct Unit {
   int nblk;        // ceil(span / 128)
 };
 
+__host__ __device__ constexpr int imin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ constexpr int imax(int a, int b) { return a > b ? a : b; }
+
 // Unit u of the launch.  Units of a batched relation are (b, h) of its
 // [B, H, N, d] tensors, right-padded to a per-batch length when lengths are
 // given; units of packed sequences are (sequence k, head h) of [1, H, N, d]
 // tensors holding the sequences back to back, sequence k on tokens
-// [cu_seqlens[k], cu_seqlens[k+1]).
-__device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
+// [cu_seqlens[k], cu_seqlens[k+1]).  `src` reads a segment's lengths and
+// sequence offsets (device memory in the kernels, host copies in the
+// schedule check).
+template <class Src>
+__host__ __device__ __forceinline__ Unit make_unit(const TcParams& p, int u, const Src& src) {
   int r = 0;
 #pragma unroll
   for (int k = 1; k < kMaxSeg; ++k)
@@ -79,17 +87,17 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
     const int k = local / s->H;
     out.b = 0;
     out.h = local - k * s->H;
-    const int a = min(max(s->cu_seqlens[k], 0), p.N);
-    const int e = min(max(s->cu_seqlens[k + 1], a), p.N);
+    const int a = imin(imax(src.cu(r, k), 0), p.N);
+    const int e = imin(imax(src.cu(r, k + 1), a), p.N);
     out.tok0 = a;
-    out.len = min(e - a, s->max_seqlen);
+    out.len = imin(e - a, s->max_seqlen);
     out.span = out.len;
     out.row0 = static_cast<long long>(out.h) * p.N + a;
   } else {
     out.b = local / s->H;
     out.h = local - out.b * s->H;
     out.tok0 = 0;
-    out.len = s->lengths ? max(0, min(p.N, s->lengths[out.b])) : p.N;
+    out.len = s->lengths ? imax(0, imin(p.N, src.len(r, out.b))) : p.N;
     out.span = p.N;
     out.row0 = (static_cast<long long>(out.b) * s->H + out.h) * p.N;
   }
@@ -97,9 +105,19 @@ __device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
   return out;
 }
 
+struct DeviceUnitSrc {
+  const TcParams& p;
+  __device__ int len(int r, int b) const { return p.seg[r].lengths[b]; }
+  __device__ int cu(int r, int k) const { return p.seg[r].cu_seqlens[k]; }
+};
+
+__device__ __forceinline__ Unit decode_unit(const TcParams& p, int u) {
+  return make_unit(p, u, DeviceUnitSrc{p});
+}
+
 // Work item -> (unit u, per-unit item index pp).  A call that covers one part
 // of the work takes the unit's items part, part + n_parts, ...
-__device__ __forceinline__ void decode_item(const TcParams& p, int item, int& u, int& pp) {
+__host__ __device__ __forceinline__ void decode_item(const TcParams& p, int item, int& u, int& pp) {
   u = item / p.n_local;
   pp = p.part + (item - u * p.n_local) * p.n_parts;
 }
@@ -107,14 +125,14 @@ __device__ __forceinline__ void decode_item(const TcParams& p, int item, int& u,
 // Row blocks of one work item: pass 0 is the longer block nblk-1-p, pass 1
 // (absent when both coincide) is block p.  An item index past the unit's
 // own pair count (a short packed sequence) has no pass.
-__device__ __forceinline__ int item_passes(const Unit& U, int pp) {
+__host__ __device__ __forceinline__ int item_passes(const Unit& U, int pp) {
   if (pp >= (U.nblk + 1) / 2) return 0;
   return (pp == U.nblk - 1 - pp) ? 1 : 2;
 }
-__device__ __forceinline__ int pass_block(const Unit& U, int pp, int pass) {
+__host__ __device__ __forceinline__ int pass_block(const Unit& U, int pp, int pass) {
   return pass == 0 ? U.nblk - 1 - pp : pp;
 }
-__device__ __forceinline__ int n_col_tiles(const TcParams& p, const Unit& U, int I) {
+__host__ __device__ __forceinline__ int n_col_tiles(const TcParams& p, const Unit& U, int I) {
   return p.causal ? I + 1 : U.nblk;
 }
 
@@ -897,12 +915,12 @@ constexpr int BN64 = 64;
 // causal mask: each off-diagonal tile then serves both orientations of its
 // entries (Z = Z^T).
 template <bool SYM>
-__device__ __forceinline__ int n_col_tiles64_s(const TcParams& p, const Unit& U, int I) {
+__host__ __device__ __forceinline__ int n_col_tiles64_s(const TcParams& p, const Unit& U, int I) {
   const int nb64 = (U.span + BN64 - 1) / BN64;
-  return (p.causal || SYM) ? min(2 * I + 2, nb64) : nb64;
+  return (p.causal || SYM) ? imin(2 * I + 2, nb64) : nb64;
 }
 template <bool SYM>
-__device__ __forceinline__ int n_col_tiles_s(const TcParams& p, const Unit& U, int I) {
+__host__ __device__ __forceinline__ int n_col_tiles_s(const TcParams& p, const Unit& U, int I) {
   return (p.causal || SYM) ? I + 1 : U.nblk;
 }
 
@@ -972,9 +990,9 @@ __device__ __forceinline__ void form_g_store(const float (&t)[NC], const float (
   }
 }
 
-__device__ __forceinline__ int n_col_tiles64(const TcParams& p, const Unit& U, int I) {
+__host__ __device__ __forceinline__ int n_col_tiles64(const TcParams& p, const Unit& U, int I) {
   const int nb64 = (U.span + BN64 - 1) / BN64;
-  return p.causal ? min(2 * I + 2, nb64) : nb64;
+  return p.causal ? imin(2 * I + 2, nb64) : nb64;
 }
 
 __global__ void __launch_bounds__(BWD_THREADS, 1)
@@ -1400,7 +1418,7 @@ constexpr int kPairMinBlocks = 33;
 constexpr int BWDP_LOGIT_WARP = 21, BWDP_GRAD_WARP = 22;
 
 // Sequence `which` (0 or 1) of pair item m: its first row block, or -1.
-__device__ __forceinline__ int pair_seq_block(const Unit& U, int m, int which) {
+__host__ __device__ __forceinline__ int pair_seq_block(const Unit& U, int m, int which) {
   const int npb = (U.nblk + 1) / 2;
   if (m >= (npb + 1) / 2) return -1;   // past a short packed sequence's items
   const int k = which == 0 ? npb - 1 - m : m;
@@ -2329,6 +2347,108 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// ----------------------------------------------------- schedule check (host)
+// The kernels' work decomposition replayed on the host: every part's work
+// items are decoded with the same helpers the kernels use, and the (unit,
+// row block, column tile) triples they visit are compared with the triples the
+// mask requires, worked out independently from row and column ranges: each
+// must be visited exactly once over the parts, no other may be, and every
+// visited tile's TMA row coordinates must lie inside the tensor.
+namespace {
+struct HostUnitSrc {
+  const int* const* lens;
+  const int* const* offs;
+  int len(int r, int b) const { return lens[r][b]; }
+  int cu(int r, int k) const { return offs[r][k]; }
+};
+}  // namespace
+
+int schedule_check(const TcParams& p0, int d, bool bwd, int n_parts, const int* const* lens,
+                   const int* const* offs, char* why, size_t why_len) {
+  const HostUnitSrc src{lens, offs};
+  auto fail = [&](const char* what, int u, int R, int J) {
+    if (why && why_len) snprintf(why, why_len, "%s (unit %d, row block %d, column tile %d)", what, u, R, J);
+    return 1;
+  };
+  // which kernel, column tile width, and whether full masks use the symmetric schedule
+  enum { FWD, TC64, PAIR, PAIR64 } kind;
+  if (!bwd) kind = FWD;
+  else if (d == 64) kind = PAIR64;
+  else if (p0.causal && p0.nblk <= kPairMinBlocks - 1) kind = TC64;
+  else kind = PAIR;
+  const int W = (kind == FWD || kind == PAIR64) ? 128 : 64;
+  const bool tri = p0.causal || (kind == PAIR || kind == PAIR64);   // lower triangle only
+  std::vector<std::vector<unsigned char>> seen(p0.n_units);
+  std::vector<Unit> units(p0.n_units);
+  for (int u = 0; u < p0.n_units; ++u) {
+    units[u] = make_unit(p0, u, src);
+    const int ncol = (units[u].span + W - 1) / W;
+    seen[u].assign(static_cast<size_t>(units[u].nblk) * (ncol > 0 ? ncol : 1), 0);
+  }
+  auto visit = [&](int u, int R, int J) -> int {
+    const Unit& U = units[u];
+    const int ncol = (U.span + W - 1) / W;
+    if (R < 0 || R >= U.nblk || J < 0 || J >= ncol) return fail("tile outside the unit", u, R, J);
+    if (U.tok0 + R * BM >= p0.N || U.tok0 + J * W >= p0.N)
+      return fail("TMA row coordinate outside the tensor", u, R, J);
+    unsigned char& c = seen[u][static_cast<size_t>(R) * ncol + J];
+    if (c) return fail("tile visited twice", u, R, J);
+    c = 1;
+    return 0;
+  };
+  for (int part = 0; part < n_parts; ++part) {
+    TcParams p = p0;
+    p.part = part;
+    p.n_parts = n_parts;
+    if (kind == PAIR || kind == PAIR64) p.n_pairs = ((p0.nblk + 1) / 2 + 1) / 2;
+    p.n_local = part < p.n_pairs ? (p.n_pairs - part + n_parts - 1) / n_parts : 0;
+    p.n_items = p.n_units * p.n_local;
+    for (int item = 0; item < p.n_items; ++item) {
+      int u, pp;
+      decode_item(p, item, u, pp);
+      if (u < 0 || u >= p.n_units) return fail("work item decodes to no unit", u, -1, -1);
+      const Unit& U = units[u];
+      if (kind == FWD || kind == TC64) {
+        for (int pass = 0; pass < item_passes(U, pp); ++pass) {
+          const int I = pass_block(U, pp, pass);
+          const int nT = kind == FWD ? n_col_tiles(p, U, I) : n_col_tiles64(p, U, I);
+          for (int J = 0; J < nT; ++J)
+            if (visit(u, I, J)) return 1;
+        }
+      } else {
+        for (int w = 0; w < 2; ++w) {
+          const int R0 = pair_seq_block(U, pp, w);
+          if (R0 < 0) break;
+          for (int rs = 0; rs < 2 && R0 + rs < U.nblk; ++rs) {
+            const int R = R0 + rs;
+            const int nT = kind == PAIR64 ? (tri ? n_col_tiles_s<true>(p, U, R)
+                                                 : n_col_tiles_s<false>(p, U, R))
+                                          : (tri ? n_col_tiles64_s<true>(p, U, R)
+                                                 : n_col_tiles64_s<false>(p, U, R));
+            for (int J = 0; J < nT; ++J)
+              if (visit(u, R, J)) return 1;
+          }
+        }
+      }
+    }
+  }
+  // every tile the mask needs: columns up to the block's last row (lower
+  // triangle), or every column
+  for (int u = 0; u < p0.n_units; ++u) {
+    const Unit& U = units[u];
+    const int ncol = (U.span + W - 1) / W;
+    for (int R = 0; R < U.nblk; ++R) {
+      const int need = tri ? imin((R * BM + BM + W - 1) / W, ncol) : ncol;
+      for (int J = 0; J < ncol; ++J) {
+        const bool got = seen[u][static_cast<size_t>(R) * ncol + J] != 0;
+        if (J < need && !got) return fail("tile never visited", u, R, J);
+        if (J >= need && got) return fail("tile outside the mask visited", u, R, J);
+      }
+    }
+  }
+  return 0;
 }
 
 // ------------------------------------------------------------ launchers

@@ -177,6 +177,23 @@ relkl_status relkl_bwd_qkv_part(int32_t n_rel, const relkl_desc* descs,
                                 float* const* dx_s, int32_t part, int32_t n_parts, void* ws,
                                 size_t ws_bytes, void* stream);
 
+/* Debug aid, host only (no GPU needed): replays the work decomposition of the
+ * tensor-core kernels that a call with these descs would launch (the forward
+ * when is_bwd is 0, else the backward the library picks), for every part of
+ * n_parts (n_parts = 1: the whole call), and checks that every (unit, row
+ * block, column tile) the mask requires is visited exactly once over the
+ * parts, that no other tile is, and that every visited tile's TMA row
+ * coordinates lie inside the tensors.  The descs' device pointers are not
+ * read: a desc with lengths or packed sequences needs HOST copies of them in
+ * host_lengths[r] / host_cu_seqlens[r] (arrays indexed by relation; may be
+ * NULL when no desc uses them).  RELKL_OK when the schedule is sound,
+ * RELKL_ERR_INVALID with a one-line reason in why (if not NULL) otherwise,
+ * RELKL_ERR_UNSUPPORTED for descs the tensor-core path does not take.        */
+relkl_status relkl_check_schedule(int32_t n_rel, const relkl_desc* descs, int32_t is_bwd,
+                                  int32_t n_parts, const int32_t* const* host_lengths,
+                                  const int32_t* const* host_cu_seqlens, char* why,
+                                  size_t why_len);
+
 /* Synchronises `stream`, then reads the workspace record.  Returns RELKL_OK
  * or RELKL_ERR_TIMEOUT; *where (if not NULL) receives the code of the wait
  * that ran out (0 when none).                                                */
