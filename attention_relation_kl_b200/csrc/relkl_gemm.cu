@@ -49,6 +49,7 @@ constexpr int MISC = BARS + NBAR * 8;
 constexpr int BYTES = MISC + 16;
 constexpr int ALLOC = BYTES + 1024;
 static_assert(ALLOC <= 232448, "GEMM shared memory exceeds 227 KB");
+static_assert(2 * BN <= 512, "TMEM columns: two 128 x 256 fp32 accumulators");
 
 constexpr int THREADS = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr unsigned long long kDrainNs = 200000000ull;

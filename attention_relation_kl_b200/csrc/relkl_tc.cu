@@ -332,6 +332,7 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
     __syncwarp();
   } else {
     // --------------------------------------------------- row warpgroups
+    static_assert(2 * 2 * BN <= 512, "TMEM columns: 2 x (Z_t, Z_s)");
     const int q = warp & 3;      // TMEM lane quarter
     const int wg = warp >> 2;    // column quarter of each tile
     const int r = q * 32 + lane;
@@ -960,6 +961,32 @@ __device__ __forceinline__ float2 sym_partner(const Unit& U, const TcParams& p, 
 // 128-byte swizzled line at row_addr.  bt, bs: -lse * log2 e of the row;
 // mul: its upstream gradient times the logit scale; entries past `lim` are 0;
 // `off`: add the transposed partner (full mask, off the diagonal block).
+// The same entries packed into NC/2 bf16 pairs in registers (for callers
+// that must wait for the G buffer after forming them).
+template <int NC>
+__device__ __forceinline__ void form_g_pack(const float (&t)[NC], const float (&s)[NC], float bt,
+                                            float bs, float mul, int col0, int lim, bool off,
+                                            const Unit& U, const TcParams& p,
+                                            uint32_t (&pk)[NC / 2]) {
+  const float2 sl2v = make_float2(p.sl2, p.sl2), btv = make_float2(bt, bt),
+               bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
+               m1 = make_float2(-1.f, -1.f);
+  const bool need_mask = col0 + NC - 1 > lim;
+#pragma unroll
+  for (int k = 0; k < NC; k += 2) {
+    const float2 zt2 = make_float2(t[k], t[k + 1]), zs2 = make_float2(s[k], s[k + 1]);
+    const float2 et = ex2_approx2(__ffma2_rn(zt2, sl2v, btv));
+    const float2 es = ex2_approx2(__ffma2_rn(zs2, sl2v, bsv));
+    float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
+    if (off) g = sym_partner(U, p, col0 + k, zt2, zs2, g);
+    if (need_mask) {
+      g.x = (col0 + k <= lim) ? g.x : 0.f;
+      g.y = (col0 + k + 1 <= lim) ? g.y : 0.f;
+    }
+    pk[k >> 1] = pack_bf16x2(g.x, g.y);
+  }
+}
+
 template <int NC>
 __device__ __forceinline__ void form_g_store(const float (&t)[NC], const float (&s)[NC],
                                              float bt, float bs, float mul, int col0, int lim,
@@ -1025,6 +1052,8 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
 
   WaitCtl wc{p.status, abort_flag, p.timeout_ns};
   constexpr uint32_t T_S = 0, T_DXI = 256, T_P = 384;
+  static_assert(T_S + 2 * 2 * BN64 <= T_DXI && T_DXI + D <= T_P && T_P + 2 * BN64 <= 512,
+                "TMEM columns: 2 x (Z_t, Z_s) | dX_I | 2 x P^T");
 
   if (threadIdx.x == 0) {
     mbar_init(FULL_I, 1);
@@ -1455,6 +1484,8 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
 
   WaitCtl wc{p.status, abort_flag, p.timeout_ns};
   constexpr uint32_t T_S = 0, T_DX0 = 128, T_P = 384;
+  static_assert(T_S + 2 * BN64 <= T_DX0 && T_DX0 + 2 * D <= T_P && T_P + 2 * BN64 <= 512,
+                "TMEM columns: Z_t, Z_s | dX_R0, dX_R1 | 2 x P^T");
 
   if (threadIdx.x == 0) {
     mbar_init(FULL_I, 1);
@@ -1819,13 +1850,19 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
             const int col0 = J * BN64 + wg * 16;
             if constexpr (SYM) {
               // full mask: tiles of the diagonal block carry G itself, the others
-              // G plus its transposed partner (4 exps per entry: the exps bound
-              // this mode, so wait for the G buffer first and store as formed)
+              // G plus its transposed partner (4 exps per entry); as in the causal
+              // path the G buffer is awaited only once the entries are formed
+              uint32_t pk[8];
+              form_g_pack<16>(t, s, btr, bsr, mr, col0, limr, J < 2 * (R0 + rs), U, p, pk);
               ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
               ok = __all_sync(0xffffffffu, ok);
               if (!ok) break;
-              form_g_store<16>(t, s, btr, bsr, mr, col0, limr, J < 2 * (R0 + rs), U, p, gsm,
-                               2 * wg, r);
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int cc = 2 * wg + h2;  // 16-byte chunk within the 128-byte row
+                st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[4 * h2], pk[4 * h2 + 1],
+                             pk[4 * h2 + 2], pk[4 * h2 + 3]);
+              }
             } else {
             const bool need_mask = col0 + 15 > limr;
             uint32_t pk[8];
@@ -1881,14 +1918,14 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
 // and its TMEM lanes are the rows j of dX[J]: the epilogue stages them row by
 // row, without a transpose.  With 64-dimensional rows the exp work per entry
 // is what bounds this kernel (2 ex2 per entry against 0.08 clk of MMA work),
-// so one logit buffer and one G buffer suffice: the next tile's logit MMAs
-// and the previous tile's gradient MMAs finish while the row warps run the
-// current tile's exps.
+// so one logit buffer suffices: the next tile's logit MMAs finish while the
+// row warps run the current tile's exps.  G is double-buffered, so the row
+// warps never wait for the previous tile's gradient MMAs before storing.
 //   TMEM: Z_t 0..127, Z_s 128..255, dX_R0 256..319, dX_R1 320..383,
 //         P 2 x 64 at 384.
 //   smem: X_t, X_s of R0 and R1 (4 x 16 KB); teacher and student column
-//         rings 2 x 16 KB each; G 32 KB (two 64-column boxes); epilogue
-//         staging 4 x 4 KB.
+//         rings 2 x 16 KB each; G 2 x 32 KB (two 64-column boxes each);
+//         epilogue staging 4 x 4 KB.
 struct BwdPair64Smem {
   static constexpr int TILE = BM * 64 * 2;           // 128 rows x 64 bf16: one box (16 KB)
   static constexpr int XT_R0 = 0;
@@ -1897,13 +1934,15 @@ struct BwdPair64Smem {
   static constexpr int XS_R1 = 3 * TILE;
   static constexpr int XT_J = 4 * TILE;              // 2 stages
   static constexpr int XS_J = XT_J + 2 * TILE;       // 2 stages
-  static constexpr int G = XS_J + 2 * TILE;          // 128 x 128 bf16, boxes of 64 columns
-  static constexpr int STG = G + 2 * TILE;           // 4 warps x one 32 x 32 f32 box
+  static constexpr int G = XS_J + 2 * TILE;          // 2 x (128 x 128 bf16, boxes of 64 columns)
+  static constexpr int G_BYTES = 2 * TILE;
+  static constexpr int STG = G + 2 * G_BYTES;        // 4 warps x one 32 x 32 f32 box
   static constexpr int STG_BYTES = 32 * 32 * 4;
   static constexpr int BARS = STG + 4 * STG_BYTES;
   // full_I, empty_I, fullT[2], emptyT[2], fullS[2], emptyS[2], s_full, s_empty,
-  // g_full, g_empty, p_full[2], p_empty[2], dxi_full, dxi_empty, drain x 2
-  static constexpr int NBAR = 22;
+  // g_full[0], g_empty[0], p_full[2], p_empty[2], dxi_full, dxi_empty, drain x 2,
+  // g_full[1], g_empty[1]
+  static constexpr int NBAR = 24;
   static constexpr int MISC = BARS + NBAR * 8;
   static constexpr int BYTES = MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
@@ -1930,7 +1969,11 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
   auto EMPTY_T = [&](int s) { return BAR(4 + s); };
   auto FULL_S = [&](int s) { return BAR(6 + s); };
   auto EMPTY_S = [&](int s) { return BAR(8 + s); };
-  const uint32_t S_FULL = BAR(10), S_EMPTY = BAR(11), G_FULL = BAR(12), G_EMPTY = BAR(13);
+  const uint32_t S_FULL = BAR(10), S_EMPTY = BAR(11);
+  // G is double-buffered: the row warps store tile t's G while the gradient
+  // MMAs of tile t-1 still read the other buffer
+  auto G_FULL = [&](int b) { return b ? BAR(22) : BAR(12); };
+  auto G_EMPTY = [&](int b) { return b ? BAR(23) : BAR(13); };
   auto P_FULL = [&](int b) { return BAR(14 + b); };
   auto P_EMPTY = [&](int b) { return BAR(16 + b); };
   const uint32_t DXI_FULL = BAR(18), DXI_EMPTY = BAR(19), DRAIN_L = BAR(20), DRAIN_G = BAR(21);
@@ -1939,6 +1982,8 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
 
   WaitCtl wc{p.status, abort_flag, p.timeout_ns};
   constexpr uint32_t T_S = 0, T_DX0 = 256, T_P = 384;
+  static_assert(T_S + 2 * BN <= T_DX0 && T_DX0 + 2 * D <= T_P && T_P + 2 * D <= 512,
+                "TMEM columns: Z_t, Z_s | dX_R0, dX_R1 | 2 x P");
 
   if (threadIdx.x == 0) {
     mbar_init(FULL_I, 1);
@@ -1953,8 +1998,10 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
     }
     mbar_init(S_FULL, 1);
     mbar_init(S_EMPTY, 16);
-    mbar_init(G_FULL, 16);
-    mbar_init(G_EMPTY, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(G_FULL(b), 16);
+      mbar_init(G_EMPTY(b), 1);
+    }
     mbar_init(DXI_FULL, 1);
     mbar_init(DXI_EMPTY, 4);
     mbar_init(DRAIN_L, 1);
@@ -2044,7 +2091,7 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
     const uint32_t dXsJ_mn0 = sw128_desc_lo(base + L::XS_J, L::TILE);
     const uint32_t dG_k = sw128_desc_lo(base + L::G, 16);
     const uint32_t dG_mn = sw128_desc_lo(base + L::G, L::TILE);
-    constexpr uint32_t J_STEP = L::TILE >> 4, BOX_STEP = L::TILE >> 4;
+    constexpr uint32_t J_STEP = L::TILE >> 4, BOX_STEP = L::TILE >> 4, G_STEP = L::G_BYTES >> 4;
     uint32_t nseq = 0, nJ = 0, nt = 0, np = 0;
     bool ok = true, issued = false;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -2088,8 +2135,8 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
             } else {
               // dX_R += G X_s[J] and P (+)= G^T X_s[R] for tile (R, J).  G_FULL
               // implies the tile's logits (hence its column tiles) are complete.
-              const int pb = np & 1;
-              if (!(ok = mbar_wait_warp(G_FULL, nt & 1, wc, W_MMA_G_FULL))) break;
+              const int pb = np & 1, gb = nt & 1;
+              if (!(ok = mbar_wait_warp(G_FULL(gb), (nt >> 1) & 1, wc, W_MMA_G_FULL))) break;
               if (first_p && !(ok = mbar_wait_warp(P_EMPTY(pb), ((np >> 1) & 1) ^ 1, wc, W_MMA_P_EMPTY)))
                 break;
               if (first_seq && !(ok = mbar_wait_warp(DXI_EMPTY, (nseq & 1) ^ 1, wc, W_MMA_DXI_EMPTY)))
@@ -2101,16 +2148,17 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
               // box every 4 steps; X_s[J] MN-major steps 16 rows (2 KB)
 #pragma unroll
               for (int k = 0; k < BN / 16; ++k)
-                umma_bf16_w_lead(lead, tmem + T_DX0 + rs * D, dG_k + (k >> 2) * BOX_STEP + (k & 3) * 2,
+                umma_bf16_w_lead(lead, tmem + T_DX0 + rs * D,
+                                 dG_k + gb * G_STEP + (k >> 2) * BOX_STEP + (k & 3) * 2,
                                  HI_1024, xsj + k * 128, HI_1024, IDESC_GX, (J > 0 || k > 0) ? 1u : 0u);
               // M = j (128, two 64-column boxes of G, LBO = box), N = c (64), K = i (128)
 #pragma unroll
               for (int k = 0; k < BM / 16; ++k)
-                umma_bf16_w_lead(lead, tmem + T_P + pb * D, dG_mn + k * 128, HI_1024,
+                umma_bf16_w_lead(lead, tmem + T_P + pb * D, dG_mn + gb * G_STEP + k * 128, HI_1024,
                                  dXsR_mn[rs] + k * 128, HI_1024, IDESC_P,
                                  (!first_p || k > 0) ? 1u : 0u);
               issued = true;
-              umma_commit_lead(lead, G_EMPTY);
+              umma_commit_lead(lead, G_EMPTY(gb));
               if (last_p) {
                 umma_commit_lead(lead, P_FULL(pb));
                 umma_commit_lead(lead, EMPTY_S(st));
@@ -2224,7 +2272,7 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
     const int r = q * 32 + lane;
     const float sl2 = p.sl2;
     // this thread's 64-byte slice of row r of G: box wg/2, chunks 4*(wg&1)..+3
-    const uint32_t gsm = base + L::G + (wg >> 1) * L::TILE + r * 128;
+    const uint32_t gsm0 = base + L::G + (wg >> 1) * L::TILE + r * 128;
     uint32_t nt = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -2269,6 +2317,7 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
             const float mr = rs ? mul[1] : mul[0];
             const int limr = rs ? lim[1] : lim[0];
             const int col0 = J * BN + wg * 32;
+            const uint32_t gsm = gsm0 + (nt & 1) * L::G_BYTES;
             if constexpr (SYM) {
               // full mask: 4 exps per entry off the diagonal tile, so the exps
               // bound this mode; the logits are read in two 16-column halves
@@ -2286,7 +2335,7 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
                   __syncwarp();
                   if (lane == 0) mbar_arrive(S_EMPTY);
                 } else {
-                  ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
+                  ok = mbar_wait(G_EMPTY(nt & 1), ((nt >> 1) & 1) ^ 1, wc, W_SM_G_EMPTY);
                   ok = __all_sync(0xffffffffu, ok);
                   if (!ok) break;
                 }
@@ -2308,7 +2357,7 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
             // the previous tile's gradient MMAs have read G (they were issued
             // a whole exp pass ago): wait first, then store each 16-byte chunk
             // as soon as it is formed, which keeps few values live at once
-            ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
+            ok = mbar_wait(G_EMPTY(nt & 1), ((nt >> 1) & 1) ^ 1, wc, W_SM_G_EMPTY);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
 #pragma unroll
@@ -2333,7 +2382,7 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(G_FULL);
+            if (lane == 0) mbar_arrive(G_FULL(nt & 1));
             ++nt;
           }
         }

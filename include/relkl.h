@@ -34,6 +34,9 @@
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
  *    only enqueue work on it and return; nothing synchronises except
  *    relkl_get_device_error().
+ *  - The current CUDA device (cudaSetDevice) must be the one that owns the
+ *    tensors and `stream`: the library reads its properties and launches on
+ *    it.
  *  - Arguments are validated before anything is enqueued; on any error code
  *    other than RELKL_OK nothing was enqueued, except RELKL_ERR_CUDA, which
  *    reports a failed launch (see relkl_last_cuda_error()).

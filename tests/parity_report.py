@@ -4,8 +4,8 @@
 
 For each case: the worst per-row KL error as a fraction of its tolerance
 (1e-3 |kl| + 1e-6), the relative error of the total KL, and the max-norm
-relative dX error against its tolerance (2e-2 for bf16 inputs, 2e-4 for the
-fp32 path).  --full adds the workload-sized cases (sampled units and rows),
+relative dX error against its tolerance (2e-2 for bf16 inputs; for the fp32
+path the per-input bound of parity.fp32_dx_tolerance).  --full adds the workload-sized cases (sampled units and rows),
 which take a few minutes of oracle time.  Needs a CUDA device.
 """
 import os
@@ -22,7 +22,7 @@ sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 import attention_relation_kl_b200 as rk  # noqa: E402
 import workload  # noqa: E402
 from oracle import dense  # noqa: E402
-from parity import DX_TOL_BF16, DX_TOL_FP32, KL_ATOL, KL_RTOL, to_np  # noqa: E402
+from parity import DX_TOL_BF16, KL_ATOL, KL_RTOL, fp32_dx_tolerance, to_np  # noqa: E402
 
 
 def margins(kl, ref_kl, dx, ref_dx, dx_tol):
@@ -47,17 +47,60 @@ def small_cases():
     return cases
 
 
+def small_cases_more():
+    """Explicit logit scale, clustered large logits (|z| ~ 70-100) and full masks
+    (the symmetric schedule)."""
+    cases = []
+    for (N, d, scale, causal) in [(4200, 128, 0.3, True), (513, 64, 0.05, False),
+                                  (150, 64, 0.3, False)]:
+        dtype = "fp32" if N == 150 else "bf16"
+        w = workload.tiny_custom(N=N, d=d, dtype=dtype, seed=N + int(1000 * scale), causal=causal)
+        xt, xs = workload.generate(w)["q"]
+        cases.append((f"scale={scale} N={N} d={d} {'causal' if causal else 'full'} {dtype}",
+                      xt, xs, causal, scale))
+    for (N, d, causal) in [(4200, 128, True), (4200, 128, False), (4300, 64, True)]:
+        xt, xs = workload.clustered_pair((1, 1, N, d), seed=N + d,
+                                         amplitude=2.5 if d == 128 else 3.0)
+        cases.append((f"large logits N={N} d={d} {'causal' if causal else 'full'} bf16",
+                       xt, xs, causal, 0.0))
+    return cases
+
+
 def run_small(out):
-    for name, xt, xs, causal in small_cases():
+    for name, xt, xs, causal, *rest in [c + (0.0,) for c in small_cases()] + small_cases_more():
+        scale = rest[0]
         gt, gs = xt.cuda(), xs.cuda()
         path = "tcgen05" if rk.relkl_path_for(gt, causal) == 1 else "CUDA-core fp32"
-        kl, st = rk.relkl_fwd(gt, gs, causal)
-        dx = rk.relkl_bwd(gt, gs, st, None, causal)
+        kl, st = rk.relkl_fwd(gt, gs, causal, scale)
+        dx = rk.relkl_bwd(gt, gs, st, None, causal, scale)
         torch.cuda.synchronize()
-        tol = DX_TOL_BF16 if path == "tcgen05" else DX_TOL_FP32
-        m = margins(to_np(kl), dense.fwd(xt, xs, causal)["kl"], to_np(dx),
-                    dense.bwd(xt, xs, None, causal), tol)
+        osc = scale if scale else None
+        tol = DX_TOL_BF16 if path == "tcgen05" else fp32_dx_tolerance(xt, xs, None, causal, osc)
+        m = margins(to_np(kl), dense.fwd(xt, xs, causal, osc)["kl"], to_np(dx),
+                    dense.bwd(xt, xs, None, causal, osc), tol)
         out.append((name, path, "all rows", *m))
+
+
+def run_packed(out):
+    """Packed variable-length sequences (garbage in the tokens of no sequence)."""
+    for lens, d, causal in [([300, 0, 1, 129, 700, 57], 128, True),
+                            ([4300, 200, 4097, 5], 128, False), ([513, 64, 1000], 64, True)]:
+        total = sum(lens) + 11
+        w = workload.tiny_custom(N=total, d=d, dtype="bf16", seed=sum(lens) + d, H=2)
+        xt, xs = workload.generate(w)["q"]
+        xt, xs = xt.clone(), xs.clone()
+        xt[:, :, total - 11:] = 30.0
+        xs[:, :, total - 11:] = -45.0
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        gcu = torch.from_numpy(cu).cuda()
+        gt, gs = xt.cuda(), xs.cuda()
+        kl, st = rk.relkl_fwd(gt, gs, causal, cu_seqlens=gcu, max_seqlen=max(lens))
+        dx = rk.relkl_bwd(gt, gs, st, None, causal, cu_seqlens=gcu, max_seqlen=max(lens))
+        torch.cuda.synchronize()
+        m = margins(to_np(kl), dense.fwd_varlen(xt, xs, cu, causal)["kl"], to_np(dx),
+                    dense.bwd_varlen(xt, xs, cu, None, causal), DX_TOL_BF16)
+        out.append((f"packed d={d} {'causal' if causal else 'full'} lengths={lens}", "tcgen05",
+                    "all rows", *m))
 
 
 def run_padded(out):
@@ -78,7 +121,8 @@ def run_padded(out):
         kl, st = rk.relkl_fwd(gt, gs, causal, lengths=gl)
         dx = rk.relkl_bwd(gt, gs, st, None, causal, lengths=gl)
         torch.cuda.synchronize()
-        tol = DX_TOL_BF16 if path == "tcgen05" else DX_TOL_FP32
+        tol = DX_TOL_BF16 if path == "tcgen05" else fp32_dx_tolerance(xt, xs, None, causal,
+                                                                       lengths=lengths)
         m = margins(to_np(kl), dense.fwd(xt, xs, causal, lengths=lengths)["kl"], to_np(dx),
                     dense.bwd(xt, xs, None, causal, lengths=lengths), tol)
         out.append((f"padded N={N} d={d} {'causal' if causal else 'full'} {dtype} lengths={lengths}",
@@ -104,9 +148,12 @@ def run_chain(out):
 
 
 def run_full(out):
+    from test_gpu_parity import _dx_rows
     for cfg, units in (("llama2_h32_n4k", [("q", 0, 0), ("v", 0, 31)]),
                        ("gqa_llama3_n16k", [("k", 0, 3), ("v", 1, 7)]),
-                       ("ext_h32_n32k", [("q", 0, 0), ("v", 0, 31)])):
+                       ("ext_h32_n32k", [("q", 0, 0), ("k", 0, 17), ("v", 0, 31)]),
+                       ("d64_h32_n32k", [("q", 0, 0), ("v", 0, 31)]),
+                       ("full_h32_n16k", [("q", 0, 5), ("v", 0, 31)])):
         w = workload.get_config(cfg)
         x = workload.generate(w)
         pairs = [(x[r][0].cuda(), x[r][1].cuda()) for r in w.relations]
@@ -117,12 +164,13 @@ def run_full(out):
         for rel, b, h in units:
             xt, xs = x[rel][0][b, h], x[rel][1][b, h]
             ref = dense.fwd_unit(xt, xs, w.causal)
-            rows = [0, 1, 127, 128, w.N // 2, w.N - 1]
+            rows = _dx_rows(w.N)
             ref_dx = dense.bwd_rows(xt, xs, rows, causal=w.causal, lse=ref)
             m = margins(to_np(outs[ri[rel]][0][b, h]), ref["kl"],
                         to_np(dxs[ri[rel]][b, h])[rows], ref_dx, DX_TOL_BF16)
             out.append((f"{cfg} unit ({rel}, b={b}, h={h})", "tcgen05 fused QKV",
-                        f"kl all {w.N} rows, dX rows {rows}", *m))
+                        f"kl all {w.N} rows, dX on {len(rows)} rows of the first, middle and "
+                        f"last work items", *m))
 
 
 def main():
@@ -130,6 +178,7 @@ def main():
     t0 = time.time()
     run_small(out)
     run_padded(out)
+    run_packed(out)
     run_chain(out)
     if "--full" in sys.argv:
         run_full(out)

@@ -113,6 +113,13 @@ def test_explicit_scale(N, d, scale, causal, path):
     dtype = "bf16" if path == 1 else "fp32"
     xt, xs = q_inputs(1, 2 if N < 1000 else 1, N, d, dtype=dtype, seed=N + int(1000 * scale),
                       causal=causal)
+    if scale * d > 20:
+        # keep the rows spread: at scale 0.3 and d = 128 unit-variance rows give a
+        # diagonal logit of ~38 against off-diagonal ones of ~3, every row is one-hot
+        # to 1e-11 and its KL (~1e-7) lies below what float32 logits of that size
+        # resolve, which would leave nothing but rounding noise to compare
+        t = xt.float() * 0.4
+        xt, xs = t.to(xt.dtype), (xs.float() * 0.4).to(xs.dtype)
     check_full(xt, xs, causal=causal, path=path, scale=scale,
                dx_tol=DX_TOL_BF16 if path == 1 else FP32)
 
