@@ -23,7 +23,11 @@
 //     stored by TMA (tiles past the matrix edge are clipped by TMA).
 // Tiles are taken M-fastest, so the CTAs that run together share the B panels
 // of a few column blocks and walk K in step, which keeps the K slices of both
-// operands in L2.  Every wait is bounded like the relation-KL kernels'.
+// operands in L2.  When the tiles would leave the last wave of SMs mostly
+// idle, K is split into `ksplit` ranges that separate work units take; their
+// partial products are then added into the zeroed dW with TMA reduce-adds
+// (two partial sums add in either order to the same float, so a split of two
+// stays deterministic).  Every wait is bounded like the relation-KL kernels'.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -61,10 +65,23 @@ struct GemmParams {
   CUtensorMap tm_b;   // dX_pre [rows, cols] bf16: dims {cols, rows}, box {64, 64}
   CUtensorMap tm_c;   // dW [D, cols] f32: dims {cols, D}, box {32, 32}, 128B swizzle
   int m_tiles, n_tiles, k_chunks;
-  int n_tiles_total;
+  int ksplit;         // K ranges per tile (1: store, >1: reduce-add into a zeroed dW)
+  int n_units;        // m_tiles * n_tiles * ksplit work units
   DevStatus* status;
   unsigned long long timeout_ns;
 };
+
+// Work unit -> (M tile, N tile, chunk range [k0, k1)).  Units of one tile's K
+// ranges are `tiles` apart, so each wave covers whole K ranges of many tiles.
+__device__ __forceinline__ void gemm_unit(const GemmParams& p, int unit, int& mt, int& nt,
+                                          int& k0, int& k1) {
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int ks = unit / tiles, tile = unit - ks * tiles;
+  mt = tile % p.m_tiles;
+  nt = tile / p.m_tiles;
+  k0 = static_cast<int>(static_cast<long long>(p.k_chunks) * ks / p.ksplit);
+  k1 = static_cast<int>(static_cast<long long>(p.k_chunks) * (ks + 1) / p.ksplit);
+}
 
 __global__ void __launch_bounds__(gemm::THREADS, 1)
 relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
@@ -116,9 +133,10 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
       uint32_t it = 0;
       uint32_t arms[STAGES] = {0, 0, 0, 0};
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.n_tiles_total; tile += gridDim.x) {
-        const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
-        for (int kc = 0; kc < p.k_chunks; ++kc, ++it) {
+      for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+        int mt, nt, k0, k1;
+        gemm_unit(p, unit, mt, nt, k0, k1);
+        for (int kc = k0; kc < k1; ++kc, ++it) {
           const int s = it % STAGES;
           if (!(ok = mbar_wait(EMPTY(s), ((it / STAGES) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
           const uint32_t a = base + s * STAGE_BYTES, b = a + A_BYTES;
@@ -148,19 +166,21 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
     constexpr uint32_t STAGE_STEP = STAGE_BYTES >> 4;
     uint32_t it = 0, nacc = 0;
     bool ok = true, issued = false;
-    for (int tile = blockIdx.x; ok && tile < p.n_tiles_total; tile += gridDim.x, ++nacc) {
+    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x, ++nacc) {
+      int mt, nt, k0, k1;
+      gemm_unit(p, unit, mt, nt, k0, k1);
       const int ab = nacc & 1;
       if (!(ok = mbar_wait_warp(ACC_EMPTY(ab), ((nacc >> 1) & 1) ^ 1, wc, W_MMA_P_EMPTY))) break;
       tc_fence_after();
       const uint32_t acc = tmem + ab * BN;
-      for (int kc = 0; kc < p.k_chunks; ++kc, ++it) {
+      for (int kc = k0; kc < k1; ++kc, ++it) {
         const int s = it % STAGES;
         if (!(ok = mbar_wait_warp(FULL(s), (it / STAGES) & 1, wc, W_MMA_FULL_J))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
           umma_bf16_w_lead(lead, acc, a0 + s * STAGE_STEP + k * 128, HI,
-                           b0 + s * STAGE_STEP + k * 128, HI, IDESC, (kc > 0 || k > 0) ? 1u : 0u);
+                           b0 + s * STAGE_STEP + k * 128, HI, IDESC, (kc > k0 || k > 0) ? 1u : 0u);
         issued = true;
         umma_commit_lead(lead, EMPTY(s));
       }
@@ -179,8 +199,9 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
     const uint32_t stg = base + STG + (warp - 2) * 2 * STG_BYTES;
     uint32_t nacc = 0, nstg = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.n_tiles_total; tile += gridDim.x, ++nacc) {
-      const int mt = tile % p.m_tiles, nt = tile / p.m_tiles;
+    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x, ++nacc) {
+      int mt, nt, k0, k1;
+      gemm_unit(p, unit, mt, nt, k0, k1);
       const int ab = nacc & 1;
       ok = mbar_wait(ACC_FULL(ab), (nacc >> 1) & 1, wc, W_EPI_P_FULL);
       ok = __all_sync(0xffffffffu, ok);
@@ -208,7 +229,10 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&p.tm_c, buf, nt * BN + c * 32, mt * BM + q * 32);
+          if (p.ksplit > 1)
+            tma_reduce_add_2d(&p.tm_c, buf, nt * BN + c * 32, mt * BM + q * 32);
+          else
+            tma_store_2d(&p.tm_c, buf, nt * BN + c * 32, mt * BM + q * 32);
           bulk_commit();
         }
         ++nstg;
@@ -266,10 +290,31 @@ int launch_wgrad(EncodeTiledFnG encode, long long rows, int D, int cols, const v
   p.m_tiles = (D + BM - 1) / BM;
   p.n_tiles = (cols + BN - 1) / BN;
   p.k_chunks = static_cast<int>((rows + BK - 1) / BK);
-  p.n_tiles_total = p.m_tiles * p.n_tiles;
+  // K split: the fraction of the SMs the last wave keeps busy, for 1..4 ranges
+  // of at least 32 chunks (2048 tokens) each; ties go to fewer ranges
+  const int tiles = p.m_tiles * p.n_tiles;
+  p.ksplit = 1;
+  double best = 0.0;
+  for (int ks = 1; ks <= 4; ++ks) {
+    if (ks > 1 && p.k_chunks / ks < 32) break;
+    const long long units = static_cast<long long>(tiles) * ks;
+    const long long waves = (units + num_sms - 1) / num_sms;
+    const double eff = static_cast<double>(units) / (static_cast<double>(waves) * num_sms);
+    if (eff > best + 0.02) {
+      best = eff;
+      p.ksplit = ks;
+    }
+  }
+  p.n_units = tiles * p.ksplit;
   p.status = status;
   p.timeout_ns = timeout_ns;
-  const int grid = p.n_tiles_total < num_sms ? p.n_tiles_total : num_sms;
+  if (p.ksplit > 1) {
+    // the partial products are reduce-added: start from zero (same stream)
+    const size_t bytes = static_cast<size_t>(D) * cols * 4;
+    cudaError_t z = cudaMemsetAsync(dw, 0, bytes, stream);
+    if (z != cudaSuccess) return static_cast<int>(z) + 2;
+  }
+  const int grid = p.n_units < num_sms ? p.n_units : num_sms;
   cudaError_t e = cudaFuncSetAttribute(relkl_wgrad_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, ALLOC);
   if (e == cudaSuccess) {

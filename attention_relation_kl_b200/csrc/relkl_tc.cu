@@ -502,27 +502,14 @@ relkl_fwd_tc_kernel(const __grid_constant__ TcParams p) {
 // =========================================================================
 //                                BACKWARD
 // =========================================================================
-template <int D>
-struct BwdSmem {
-  static constexpr int TILE = BM * D * 2;
-  static constexpr int XT_I = 0;
-  static constexpr int XS_I = TILE;
-  static constexpr int XT_R = 2 * TILE;            // teacher column tile, one stage
-  static constexpr int XS_R = 3 * TILE;            // student ring, two stages
-  static constexpr int G = 5 * TILE;               // 128 x 128 bf16 gradient tile (two boxes)
-  static constexpr int STG = G + 2 * BOX;          // epilogue staging: 4 warps x 2 x 4 KB
-  static constexpr int STG_BYTES = 32 * 32 * 4;    // one 32-row x 32-col f32 box
-  static constexpr int BARS = STG + 4 * 2 * STG_BYTES;
-  // full_I, empty_I, fullT, emptyT, fullS[2], emptyS[2], s_full, s_empty,
-  // g_full, g_empty, p_full, p_empty, dxi_full, dxi_empty, drain
-  static constexpr int NBAR = 17;
-  static constexpr int MISC = BARS + NBAR * 8;
-  static constexpr int BYTES = MISC + 16;
-  static constexpr int ALLOC = BYTES + 1024;
-};
-
-// Warps 0-15: four row warpgroups (columns [32k, 32k+32) of every tile);
-// warps 16-19: epilogue; warp 20: TMA; warp 21: MMA.
+// Phase 2 on the pages: recompute the logit tiles, rebuild R_t and R_s from
+// the stored LSEs, form G = dkl (R_s - R_t) (bf16, in shared memory) and
+// stream it into dX_s = s (G X_s[J] for the row block, G^T X_s[I] for the
+// column block).  Three kernels share the work: one 128-row block per pass
+// (d = 128, causal, few row blocks), adjacent row-block pairs (d = 128
+// otherwise) and adjacent pairs with 128-column tiles (d = 64).
+// Warps 0-15: four row warpgroups; warps 16-19: epilogue; warp 20: TMA;
+// warp 21 (and 22 in the paired kernels): MMA.
 constexpr int BWD_THREADS = 704;
 constexpr int BWD_EPI_WARP = 16, BWD_TMA_WARP = 20, BWD_MMA_WARP = 21;
 
@@ -563,322 +550,10 @@ __device__ __forceinline__ void epilogue_reduce(uint32_t taddr, uint32_t stg, ui
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(BWD_THREADS, 1)
-relkl_bwd_tc_kernel(const __grid_constant__ TcParams p) {
-  using L = BwdSmem<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  const uint32_t bar0 = base + L::BARS;
-  auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
-  const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1), FULL_T = BAR(2), EMPTY_T = BAR(3);
-  auto FULL_S = [&](int s) { return BAR(4 + s); };
-  auto EMPTY_S = [&](int s) { return BAR(6 + s); };
-  const uint32_t S_FULL = BAR(8), S_EMPTY = BAR(9), G_FULL = BAR(10), G_EMPTY = BAR(11);
-  const uint32_t P_FULL = BAR(12), P_EMPTY = BAR(13), DXI_FULL = BAR(14), DXI_EMPTY = BAR(15);
-  const uint32_t DRAIN = BAR(16);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
-
-  WaitCtl wc{p.status, abort_flag, p.timeout_ns};
-
-  // TMEM columns
-  constexpr uint32_t T_ST = 0, T_SS = 128, T_DXI = 256, T_P = 256 + D;
-
-  if (threadIdx.x == 0) {
-    mbar_init(FULL_I, 1);
-    mbar_init(EMPTY_I, 1);
-    mbar_init(FULL_T, 1);
-    mbar_init(EMPTY_T, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(FULL_S(s), 1);
-      mbar_init(EMPTY_S(s), 1);
-    }
-    mbar_init(S_FULL, 1);
-    mbar_init(S_EMPTY, 16);
-    mbar_init(G_FULL, 16);
-    mbar_init(G_EMPTY, 1);
-    mbar_init(P_FULL, 1);
-    mbar_init(P_EMPTY, 4);
-    mbar_init(DXI_FULL, 1);
-    mbar_init(DXI_EMPTY, 4);
-    mbar_init(DRAIN, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == BWD_MMA_WARP) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == BWD_TMA_WARP) {
-    // ------------------------------------------------------------ TMA
-    if (lane == 0) {
-      for (int s = 0; s < p.n_seg; ++s) {
-        tma_prefetch_desc(&p.seg[s].tm_t);
-        tma_prefetch_desc(&p.seg[s].tm_s);
-        tma_prefetch_desc(&p.seg[s].tm_dx);
-      }
-      uint32_t nI = 0, nJ = 0, armsT = 0;
-      uint32_t armsS[2] = {0, 0};   // loads issued per ring stage
-      bool ok = true;
-      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        int u, pp;
-        decode_item(p, item, u, pp);
-        const Unit U = decode_unit(p, u);
-        for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
-          const int I = pass_block(U, pp, pass);
-          if (!(ok = mbar_wait(EMPTY_I, (nI & 1) ^ 1, wc, W_TMA_EMPTY_I))) break;
-          mbar_arrive_expect_tx(FULL_I, 2 * L::TILE);
-#pragma unroll
-          for (int b = 0; b < D / 64; ++b) {
-            tma_load_4d(base + L::XT_I + b * BOX, &U.seg->tm_t, FULL_I, b * 64, U.tok0 + I * BM, U.h, U.b);
-            tma_load_4d(base + L::XS_I + b * BOX, &U.seg->tm_s, FULL_I, b * 64, U.tok0 + I * BM, U.h, U.b);
-          }
-          ++nI;
-          const int nT = n_col_tiles(p, U, I);
-          for (int J = 0; J < nT; ++J) {
-            // teacher tile first: its single slot frees as soon as Z_t(J-1) is done,
-            // while a student slot frees only after the gradient MMAs of J-2
-            if (!(ok = mbar_wait(EMPTY_T, (nJ & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
-            mbar_arrive_expect_tx(FULL_T, L::TILE);
-#pragma unroll
-            for (int b = 0; b < D / 64; ++b)
-              tma_load_4d(base + L::XT_R + b * BOX, &U.seg->tm_t, FULL_T, b * 64, U.tok0 + J * BN,
-                          U.h, U.b);
-            ++armsT;
-            const int st = nJ & 1;
-            if (!(ok = mbar_wait(EMPTY_S(st), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
-            mbar_arrive_expect_tx(FULL_S(st), L::TILE);
-#pragma unroll
-            for (int b = 0; b < D / 64; ++b)
-              tma_load_4d(base + L::XS_R + st * L::TILE + b * BOX, &U.seg->tm_s, FULL_S(st),
-                          b * 64, U.tok0 + J * BN, U.h, U.b);
-            ++armsS[st];
-            ++nJ;
-          }
-        }
-      }
-      // wait for the copies still in flight before the CTA may exit
-      if (nI) mbar_wait_drain(FULL_I, (nI - 1) & 1, kDrainNs);
-      if (armsT) mbar_wait_drain(FULL_T, (armsT - 1) & 1, kDrainNs);
-      for (int st = 0; st < 2; ++st)
-        if (armsS[st]) mbar_wait_drain(FULL_S(st), (armsS[st] - 1) & 1, kDrainNs);
-    }
-    __syncwarp();
-  } else if (warp == BWD_MMA_WARP) {
-    // ------------------------------------------------------------ MMA
-    if (lane == 0) {
-      constexpr uint32_t IDESC_GX = idesc_bf16_f32(BM, D, 0, 1);   // A = G (K-major), B = X (MN)
-      constexpr uint32_t IDESC_GTX = idesc_bf16_f32(BM, D, 1, 1);  // A = G^T (MN), B = X (MN)
-      uint32_t nI = 0, nJ = 0, ns = 0, ng = 0, nrb = 0;
-      bool ok = true, issued = false;
-      // gradient MMAs of the tile that used ring stage `st`; `first` starts dX_I
-      auto grad = [&](int st, bool first) -> bool {
-        if (!mbar_wait(G_FULL, ng & 1, wc, W_MMA_G_FULL)) return false;
-        if (!mbar_wait(P_EMPTY, (ng & 1) ^ 1, wc, W_MMA_P_EMPTY)) return false;
-        if (first && !mbar_wait(DXI_EMPTY, (nrb & 1) ^ 1, wc, W_MMA_DXI_EMPTY)) return false;
-        tc_fence_after();
-        const uint32_t g = base + L::G;
-        const uint32_t xsj = base + L::XS_R + st * L::TILE;
-        const uint32_t xsi = base + L::XS_I;
-        // dX_I += G X_s[J]: M = i, N = c, K = j
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
-          const uint64_t ad = sw128_desc(g + (k >> 2) * BOX + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = sw128_desc(xsj + k * 2048, BOX, 1024);
-          umma_bf16(tmem + T_DXI, ad, bd, IDESC_GX, (!first || k > 0) ? 1u : 0u);
-        }
-        // P = G^T X_s[I]: M = j, N = c, K = i
-#pragma unroll
-        for (int k = 0; k < BM / 16; ++k) {
-          const uint64_t ad = sw128_desc(g + k * 2048, BOX, 1024);
-          const uint64_t bd = sw128_desc(xsi + k * 2048, BOX, 1024);
-          umma_bf16(tmem + T_P, ad, bd, IDESC_GTX, k > 0 ? 1u : 0u);
-        }
-        umma_commit(G_EMPTY);
-        umma_commit(P_FULL);
-        umma_commit(EMPTY_S(st));
-        ++ng;
-        return true;
-      };
-      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        int u, pp;
-        decode_item(p, item, u, pp);
-        const Unit U = decode_unit(p, u);
-        for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
-          const int I = pass_block(U, pp, pass);
-          if (!(ok = mbar_wait(FULL_I, nI & 1, wc, W_MMA_FULL_I))) break;
-          const int nT = n_col_tiles(p, U, I);
-          int prev_st = -1;
-          for (int J = 0; J < nT; ++J) {
-            const int st = nJ & 1;
-            if (!(ok = mbar_wait(FULL_T, nJ & 1, wc, W_MMA_FULL_J))) break;
-            if (!(ok = mbar_wait(S_EMPTY, (ns & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
-            tc_fence_after();
-            issue_logits<D>(tmem + T_ST, base + L::XT_I, base + L::XT_R);
-            issued = true;
-            umma_commit(EMPTY_T);   // the teacher tile is free as soon as Z_t is done
-            if (!(ok = mbar_wait(FULL_S(st), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
-            tc_fence_after();
-            issue_logits<D>(tmem + T_SS, base + L::XS_I, base + L::XS_R + st * L::TILE);
-            umma_commit(S_FULL);
-            ++ns;
-            ++nJ;
-            if (prev_st >= 0 && !(ok = grad(prev_st, J == 1))) break;
-            prev_st = st;
-          }
-          if (!ok) break;
-          if (!(ok = grad(prev_st, nT == 1))) break;
-          umma_commit(EMPTY_I);
-          umma_commit(DXI_FULL);
-          ++nI;
-          ++nrb;
-        }
-      }
-      if (issued) {
-        umma_commit(DRAIN);
-        mbar_wait_drain(DRAIN, 0, kDrainNs);
-      }
-    }
-    __syncwarp();
-  } else if (warp >= BWD_EPI_WARP) {
-    // ------------------------------------------------------- epilogue
-    const int q = warp - BWD_EPI_WARP;
-    const uint32_t stg = base + L::STG + q * 2 * L::STG_BYTES;
-    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-    uint32_t np = 0, nrb = 0, nstg = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      int u, pp;
-        decode_item(p, item, u, pp);
-      const Unit U = decode_unit(p, u);
-      for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
-        const int I = pass_block(U, pp, pass);
-        const int nT = n_col_tiles(p, U, I);
-        for (int J = 0; J < nT; ++J) {
-          ok = mbar_wait(P_FULL, np & 1, wc, W_EPI_P_FULL);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-          epilogue_reduce<D>(tmem + lane_addr + T_P, stg, nstg, &U.seg->tm_dx, U.tok0 + J * BN + q * 32,
-                             U.h, U.b, p.N, lane, P_EMPTY);
-          ++np;
-        }
-        if (!ok) break;
-        ok = mbar_wait(DXI_FULL, nrb & 1, wc, W_EPI_DXI_FULL);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        epilogue_reduce<D>(tmem + lane_addr + T_DXI, stg, nstg, &U.seg->tm_dx, U.tok0 + I * BM + q * 32,
-                           U.h, U.b, p.N, lane, DXI_EMPTY);
-        ++nrb;
-      }
-    }
-    if (lane == 0) bulk_wait_all();   // reduces must finish reading staging before exit
-    __syncwarp();
-  } else {
-    // --------------------------------------------------- row warpgroups
-    const int q = warp & 3;
-    const int wg = warp >> 2;      // column quarter of each tile
-    const int r = q * 32 + lane;
-    const float sl2 = p.sl2;
-    // this thread's 64-byte slice of row r of the G tile: box wg/2, chunks 4*(wg&1)..+3
-    const uint32_t gsm = base + L::G + (wg >> 1) * BOX + r * 128;
-    uint32_t ns = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-      int u, pp;
-        decode_item(p, item, u, pp);
-      const Unit U = decode_unit(p, u);
-      for (int pass = 0; ok && pass < item_passes(U, pp); ++pass) {
-        const int I = pass_block(U, pp, pass);
-        const int row = I * BM + r;
-        const int L = U.len;
-        const bool rvalid = row < L;
-        float bt = 0.f, bs = 0.f, mul = 0.f;
-        if (rvalid) {
-          const float4 st4 = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + row];
-          bt = -st4.y * kLog2e;
-          bs = -st4.z * kLog2e;
-          const float up = U.seg->dkl ? U.seg->dkl[U.row0 + row] : 1.0f / static_cast<float>(L);
-          mul = up * p.scale;   // the logit scale of dX_s is folded into G
-        }
-        const int lim = !rvalid ? -1 : (p.causal ? min(row, L - 1) : L - 1);
-        const int nT = n_col_tiles(p, U, I);
-        for (int J = 0; J < nT; ++J) {
-          ok = mbar_wait(S_FULL, ns & 1, wc, W_SM_S_FULL);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + wg * 32;
-          float t[32], s[32];
-          tmem_ld32(ta + T_ST, t);
-          tmem_ld32(ta + T_SS, s);
-          tmem_wait_ld();
-          // hand the logit tiles back at once: the next tile's MMAs overlap this one
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(S_EMPTY);
-          const int col0 = J * BN + wg * 32;
-          const bool need_mask = !rvalid || (col0 + 31 > lim);
-          uint32_t pk[16];
-          const float2 sl2v = make_float2(sl2, sl2), btv = make_float2(bt, bt),
-                       bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
-                       m1 = make_float2(-1.f, -1.f);
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
-            const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
-            const float2 et = ex2_approx2(at), es = ex2_approx2(as);
-            float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
-            if (need_mask) {
-              g.x = (col0 + k <= lim) ? g.x : 0.f;
-              g.y = (col0 + k + 1 <= lim) ? g.y : 0.f;
-            }
-            pk[k >> 1] = pack_bf16x2(g.x, g.y);
-          }
-          // the G buffer is free once the previous tile's gradient MMAs completed
-          ok = mbar_wait(G_EMPTY, (ns & 1) ^ 1, wc, W_SM_G_EMPTY);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int cc = (wg & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
-            st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2],
-                         pk[4 * q4 + 3]);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(G_FULL);
-          ++ns;
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == BWD_MMA_WARP) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
 // =========================================================================
 //              BACKWARD, d = 128: 64-column tiles, double-buffered
 // =========================================================================
-// Same mathematics as relkl_bwd_tc_kernel with column tiles of 64: the logit
+// One 128-row block per pass with column tiles of 64: the logit
 // tiles (2 x 64 TMEM columns), the gradient tile G (16 KB) and the transposed
 // column-side product P^T = X_s[I]^T G (64 TMEM columns, M = d = 128) are all
 // double-buffered, and the student column tiles pass through a 4-stage ring, so
@@ -928,45 +603,44 @@ __host__ __device__ __forceinline__ int n_col_tiles_s(const TcParams& p, const U
 // Row-side G plus, for an entry (i, j) off the diagonal block of a full mask,
 // its transposed partner G(j, i) = dkl_j (R_s - R_t)(j, i), which reuses the
 // logits because Z(j, i) = Z(i, j).  Row j's LSEs and upstream gradient come
-// from the statistics of column j.  Adds the partners of columns c, c+1
-// (local to the unit) to g; zt2 / zs2 are the raw logit accumulators of the
-// pair.
-__device__ __forceinline__ float2 sym_partner(const Unit& U, const TcParams& p, int c, float2 zt2,
+// from the statistics of column j: before the tile's logits arrive, lane l of
+// each warp loads the constants of one of the warp's columns
+// (partner_column), and the entries take them from that lane by shuffles.
+struct PartnerCol {
+  float bt, bs, mul;   // -lse_t log2 e, -lse_s log2 e, dkl * scale of one column
+};
+
+__device__ __forceinline__ PartnerCol partner_column(const Unit& U, const TcParams& p, int c) {
+  const int cc = imin(c, U.span - 1);   // columns past the unit are masked; keep the load inside
+  const float4 a = reinterpret_cast<const float4*>(U.seg->stats)[U.row0 + cc];
+  PartnerCol out;
+  out.bt = -a.y * kLog2e;
+  out.bs = -a.z * kLog2e;
+  out.mul = (U.seg->dkl ? U.seg->dkl[U.row0 + cc] : 1.0f / static_cast<float>(U.len)) * p.scale;
+  return out;
+}
+
+// Adds the partners of the column pair held by lanes src, src + 1 to g; zt2 /
+// zs2 are the raw logit accumulators of the pair.
+__device__ __forceinline__ float2 sym_partner(const PartnerCol& pc, int src, float sl2, float2 zt2,
                                               float2 zs2, float2 g) {
-  // keep this pair's loads next to their use: hoisting all of a tile's column
-  // statistics ahead of the exps would not fit the row warps' registers
-  __syncwarp();
-  const float4* st = reinterpret_cast<const float4*>(U.seg->stats) + U.row0;
-  const int last = U.span - 1;
-  const int c0 = min(c, last), c1 = min(c + 1, last);
-  const float4 a = st[c0], b = st[c1];
-  const float2 btc = make_float2(-a.y * kLog2e, -b.y * kLog2e);
-  const float2 bsc = make_float2(-a.z * kLog2e, -b.z * kLog2e);
-  float2 mulc;
-  if (U.seg->dkl) {
-    const float* dk = U.seg->dkl + U.row0;
-    mulc = make_float2(dk[c0] * p.scale, dk[c1] * p.scale);
-  } else {
-    const float m = p.scale / static_cast<float>(U.len);
-    mulc = make_float2(m, m);
-  }
-  const float2 sl2v = make_float2(p.sl2, p.sl2);
+  constexpr unsigned kAll = 0xffffffffu;
+  const float2 btc = make_float2(__shfl_sync(kAll, pc.bt, src), __shfl_sync(kAll, pc.bt, src + 1));
+  const float2 bsc = make_float2(__shfl_sync(kAll, pc.bs, src), __shfl_sync(kAll, pc.bs, src + 1));
+  const float2 mulc =
+      make_float2(__shfl_sync(kAll, pc.mul, src), __shfl_sync(kAll, pc.mul, src + 1));
+  const float2 sl2v = make_float2(sl2, sl2);
   const float2 et = ex2_approx2(__ffma2_rn(zt2, sl2v, btc));
   const float2 es = ex2_approx2(__ffma2_rn(zs2, sl2v, bsc));
   return __ffma2_rn(__ffma2_rn(et, make_float2(-1.f, -1.f), es), mulc, g);
 }
 
-// Forms NC consecutive entries of one row of the bf16 gradient tile and
-// stores them as NC/8 16-byte chunks (chunk0, chunk0 + 1, ...) of the row's
-// 128-byte swizzled line at row_addr.  bt, bs: -lse * log2 e of the row;
-// mul: its upstream gradient times the logit scale; entries past `lim` are 0;
-// `off`: add the transposed partner (full mask, off the diagonal block).
 // The same entries packed into NC/2 bf16 pairs in registers (for callers
 // that must wait for the G buffer after forming them).
 template <int NC>
 __device__ __forceinline__ void form_g_pack(const float (&t)[NC], const float (&s)[NC], float bt,
                                             float bs, float mul, int col0, int lim, bool off,
-                                            const Unit& U, const TcParams& p,
+                                            const PartnerCol& pc, int lane0, const TcParams& p,
                                             uint32_t (&pk)[NC / 2]) {
   const float2 sl2v = make_float2(p.sl2, p.sl2), btv = make_float2(bt, bt),
                bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
@@ -978,7 +652,7 @@ __device__ __forceinline__ void form_g_pack(const float (&t)[NC], const float (&
     const float2 et = ex2_approx2(__ffma2_rn(zt2, sl2v, btv));
     const float2 es = ex2_approx2(__ffma2_rn(zs2, sl2v, bsv));
     float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
-    if (off) g = sym_partner(U, p, col0 + k, zt2, zs2, g);
+    if (off) g = sym_partner(pc, lane0 + k, p.sl2, zt2, zs2, g);
     if (need_mask) {
       g.x = (col0 + k <= lim) ? g.x : 0.f;
       g.y = (col0 + k + 1 <= lim) ? g.y : 0.f;
@@ -990,8 +664,9 @@ __device__ __forceinline__ void form_g_pack(const float (&t)[NC], const float (&
 template <int NC>
 __device__ __forceinline__ void form_g_store(const float (&t)[NC], const float (&s)[NC],
                                              float bt, float bs, float mul, int col0, int lim,
-                                             bool off, const Unit& U, const TcParams& p,
-                                             uint32_t row_addr, int chunk0, int r) {
+                                             bool off, const PartnerCol& pc, int lane0,
+                                             const TcParams& p, uint32_t row_addr, int chunk0,
+                                             int r) {
   const float2 sl2v = make_float2(p.sl2, p.sl2), btv = make_float2(bt, bt),
                bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
                m1 = make_float2(-1.f, -1.f);
@@ -1006,7 +681,7 @@ __device__ __forceinline__ void form_g_store(const float (&t)[NC], const float (
       const float2 et = ex2_approx2(__ffma2_rn(zt2, sl2v, btv));
       const float2 es = ex2_approx2(__ffma2_rn(zs2, sl2v, bsv));
       float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
-      if (off) g = sym_partner(U, p, col0 + k, zt2, zs2, g);
+      if (off) g = sym_partner(pc, lane0 + k, p.sl2, zt2, zs2, g);
       if (need_mask) {
         g.x = (col0 + k <= lim) ? g.x : 0.f;
         g.y = (col0 + k + 1 <= lim) ? g.y : 0.f;
@@ -1830,6 +1505,12 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
           for (int rs = 0; rs < 2; ++rs) {
             if (rs == 0 && J >= nT0) continue;
             if (rs == 1 && !has1) continue;
+            // full mask, off the diagonal block: each lane fetches the partner
+            // constants of one of this warpgroup's 16 columns while the logits
+            // are still being computed
+            const bool off = SYM && J < 2 * (R0 + rs);
+            PartnerCol pc{0.f, 0.f, 0.f};
+            if (off) pc = partner_column(U, p, J * BN64 + wg * 16 + (lane & 15));
             ok = mbar_wait(S_FULL, nt & 1, wc, W_SM_S_FULL);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -1853,7 +1534,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
               // G plus its transposed partner (4 exps per entry); as in the causal
               // path the G buffer is awaited only once the entries are formed
               uint32_t pk[8];
-              form_g_pack<16>(t, s, btr, bsr, mr, col0, limr, J < 2 * (R0 + rs), U, p, pk);
+              form_g_pack<16>(t, s, btr, bsr, mr, col0, limr, off, pc, 0, p, pk);
               ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
               ok = __all_sync(0xffffffffu, ok);
               if (!ok) break;
@@ -2308,6 +1989,12 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
           for (int rs = 0; rs < 2; ++rs) {
             if (rs == 0 && J >= nT0) continue;
             if (rs == 1 && !has1) continue;
+            // full mask, off the diagonal tile: each lane fetches the partner
+            // constants of one of this warpgroup's 32 columns while the logits
+            // are still being computed
+            const bool off = SYM && J < R0 + rs;
+            PartnerCol pc{0.f, 0.f, 0.f};
+            if (off) pc = partner_column(U, p, J * BN + wg * 32 + lane);
             ok = mbar_wait(S_FULL, nt & 1, wc, W_SM_S_FULL);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -2318,68 +2005,32 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
             const int limr = rs ? lim[1] : lim[0];
             const int col0 = J * BN + wg * 32;
             const uint32_t gsm = gsm0 + (nt & 1) * L::G_BYTES;
-            if constexpr (SYM) {
-              // full mask: 4 exps per entry off the diagonal tile, so the exps
-              // bound this mode; the logits are read in two 16-column halves
-              // (the second half releases the buffer) to keep registers free
-              // for the partners' statistics
-              const bool off = J < R0 + rs;
+            // the logits are read in two 16-column halves, each turned into G and
+            // stored before the next is loaded (the second half releases the
+            // buffer): few values live at once, and the exps, which bound this
+            // kernel, leave time for the next tile's logit MMAs either way.  A
+            // full mask adds the transposed partners off the diagonal tile
+            // (4 exps per entry).
 #pragma unroll 1
-              for (int hf = 0; hf < 2; ++hf) {
-                float t[16], s[16];
-                tmem_ld16(ta + hf * 16, t);
-                tmem_ld16(ta + BN + hf * 16, s);
-                tmem_wait_ld();
-                if (hf == 1) {
-                  tc_fence_before();
-                  __syncwarp();
-                  if (lane == 0) mbar_arrive(S_EMPTY);
-                } else {
-                  ok = mbar_wait(G_EMPTY(nt & 1), ((nt >> 1) & 1) ^ 1, wc, W_SM_G_EMPTY);
-                  ok = __all_sync(0xffffffffu, ok);
-                  if (!ok) break;
-                }
-                form_g_store<16>(t, s, btr, bsr, mr, col0 + hf * 16, limr, off, U, p, gsm,
-                                 (wg & 1) * 4 + hf * 2, r);
+            for (int hf = 0; hf < 2; ++hf) {
+              float t[16], s[16];
+              tmem_ld16(ta + hf * 16, t);
+              tmem_ld16(ta + BN + hf * 16, s);
+              tmem_wait_ld();
+              if (hf == 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(S_EMPTY);
+              } else {
+                // the gradient MMAs of two tiles back have read this G buffer
+                ok = mbar_wait(G_EMPTY(nt & 1), ((nt >> 1) & 1) ^ 1, wc, W_SM_G_EMPTY);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
               }
-              if (!ok) break;
-            } else {
-            float t[32], s[32];
-            tmem_ld32(ta, t);
-            tmem_ld32(ta + BN, s);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(S_EMPTY);
-            const float2 btv = make_float2(btr, btr), bsv = make_float2(bsr, bsr),
-                         mulv = make_float2(mr, mr);
-            const bool need_mask = col0 + 31 > limr;
-            // the previous tile's gradient MMAs have read G (they were issued
-            // a whole exp pass ago): wait first, then store each 16-byte chunk
-            // as soon as it is formed, which keeps few values live at once
-            ok = mbar_wait(G_EMPTY(nt & 1), ((nt >> 1) & 1) ^ 1, wc, W_SM_G_EMPTY);
-            ok = __all_sync(0xffffffffu, ok);
+              form_g_store<16>(t, s, btr, bsr, mr, col0 + hf * 16, limr, off, pc, hf * 16, p, gsm,
+                               (wg & 1) * 4 + hf * 2, r);
+            }
             if (!ok) break;
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              uint32_t pk[4];
-#pragma unroll
-              for (int k2 = 0; k2 < 8; k2 += 2) {
-                const int k = q4 * 8 + k2;
-                const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
-                const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
-                const float2 et = ex2_approx2(at), es = ex2_approx2(as);
-                float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
-                if (need_mask) {
-                  g.x = (col0 + k <= limr) ? g.x : 0.f;
-                  g.y = (col0 + k + 1 <= limr) ? g.y : 0.f;
-                }
-                pk[k2 >> 1] = pack_bf16x2(g.x, g.y);
-              }
-              const int cc = (wg & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
-              st_shared_v4(gsm + ((cc ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
-            }
-            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(G_FULL(nt & 1));
@@ -2409,8 +2060,9 @@ namespace {
 struct HostUnitSrc {
   const int* const* lens;
   const int* const* offs;
-  int len(int r, int b) const { return lens[r][b]; }
-  int cu(int r, int k) const { return offs[r][k]; }
+  // host copies; declared for both sides only because make_unit is
+  __host__ __device__ int len(int r, int b) const { return lens[r][b]; }
+  __host__ __device__ int cu(int r, int k) const { return offs[r][k]; }
 };
 }  // namespace
 
@@ -2508,16 +2160,6 @@ static cudaError_t launch_fwd(const TcParams& p, int grid, cudaStream_t stream) 
                                        FwdSmem<D>::ALLOC);
   if (e != cudaSuccess) return e;
   k<<<grid, FWD_THREADS, FwdSmem<D>::ALLOC, stream>>>(p);
-  return cudaGetLastError();
-}
-
-template <int D>
-static cudaError_t launch_bwd(const TcParams& p, int grid, cudaStream_t stream) {
-  auto k = relkl_bwd_tc_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       BwdSmem<D>::ALLOC);
-  if (e != cudaSuccess) return e;
-  k<<<grid, BWD_THREADS, BwdSmem<D>::ALLOC, stream>>>(p);
   return cudaGetLastError();
 }
 
