@@ -153,17 +153,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
       : "memory");
 }
 
-// 2-D tiled reduce-add of one shared-memory box into global memory (f32 add
-// performed at L2); elements outside the tensor are skipped.
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int c0,
-                                                  int c1) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group"
-      " [%0, {%2, %3}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(c0), "r"(c1)
-      : "memory");
-}
-
 // 4-D tiled reduce-add of one shared-memory box into global memory (f32 add
 // performed at L2).  Elements outside the tensor are skipped.  Completion is
 // tracked by this thread's bulk async-groups.

@@ -23,11 +23,7 @@
 //     stored by TMA (tiles past the matrix edge are clipped by TMA).
 // Tiles are taken M-fastest, so the CTAs that run together share the B panels
 // of a few column blocks and walk K in step, which keeps the K slices of both
-// operands in L2.  When the tiles would leave the last wave of SMs mostly
-// idle, K is split into `ksplit` ranges that separate work units take; their
-// partial products are then added into the zeroed dW with TMA reduce-adds
-// (two partial sums add in either order to the same float, so a split of two
-// stays deterministic).  Every wait is bounded like the relation-KL kernels'.
+// operands in L2.  Every wait is bounded like the relation-KL kernels'.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -65,22 +61,18 @@ struct GemmParams {
   CUtensorMap tm_b;   // dX_pre [rows, cols] bf16: dims {cols, rows}, box {64, 64}
   CUtensorMap tm_c;   // dW [D, cols] f32: dims {cols, D}, box {32, 32}, 128B swizzle
   int m_tiles, n_tiles, k_chunks;
-  int ksplit;         // K ranges per tile (1: store, >1: reduce-add into a zeroed dW)
-  int n_units;        // m_tiles * n_tiles * ksplit work units
+  int n_units;        // m_tiles * n_tiles output tiles
   DevStatus* status;
   unsigned long long timeout_ns;
 };
 
-// Work unit -> (M tile, N tile, chunk range [k0, k1)).  Units of one tile's K
-// ranges are `tiles` apart, so each wave covers whole K ranges of many tiles.
+// Work unit -> (M tile, N tile, chunk range [k0, k1)): M-fastest tiles, all of K.
 __device__ __forceinline__ void gemm_unit(const GemmParams& p, int unit, int& mt, int& nt,
                                           int& k0, int& k1) {
-  const int tiles = p.m_tiles * p.n_tiles;
-  const int ks = unit / tiles, tile = unit - ks * tiles;
-  mt = tile % p.m_tiles;
-  nt = tile / p.m_tiles;
-  k0 = static_cast<int>(static_cast<long long>(p.k_chunks) * ks / p.ksplit);
-  k1 = static_cast<int>(static_cast<long long>(p.k_chunks) * (ks + 1) / p.ksplit);
+  mt = unit % p.m_tiles;
+  nt = unit / p.m_tiles;
+  k0 = 0;
+  k1 = p.k_chunks;
 }
 
 __global__ void __launch_bounds__(gemm::THREADS, 1)
@@ -229,10 +221,7 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (p.ksplit > 1)
-            tma_reduce_add_2d(&p.tm_c, buf, nt * BN + c * 32, mt * BM + q * 32);
-          else
-            tma_store_2d(&p.tm_c, buf, nt * BN + c * 32, mt * BM + q * 32);
+          tma_store_2d(&p.tm_c, buf, nt * BN + c * 32, mt * BM + q * 32);
           bulk_commit();
         }
         ++nstg;
@@ -290,30 +279,9 @@ int launch_wgrad(EncodeTiledFnG encode, long long rows, int D, int cols, const v
   p.m_tiles = (D + BM - 1) / BM;
   p.n_tiles = (cols + BN - 1) / BN;
   p.k_chunks = static_cast<int>((rows + BK - 1) / BK);
-  // K split: the fraction of the SMs the last wave keeps busy, for 1..4 ranges
-  // of at least 32 chunks (2048 tokens) each; ties go to fewer ranges
-  const int tiles = p.m_tiles * p.n_tiles;
-  p.ksplit = 1;
-  double best = 0.0;
-  for (int ks = 1; ks <= 4; ++ks) {
-    if (ks > 1 && p.k_chunks / ks < 32) break;
-    const long long units = static_cast<long long>(tiles) * ks;
-    const long long waves = (units + num_sms - 1) / num_sms;
-    const double eff = static_cast<double>(units) / (static_cast<double>(waves) * num_sms);
-    if (eff > best + 0.02) {
-      best = eff;
-      p.ksplit = ks;
-    }
-  }
-  p.n_units = tiles * p.ksplit;
+  p.n_units = p.m_tiles * p.n_tiles;
   p.status = status;
   p.timeout_ns = timeout_ns;
-  if (p.ksplit > 1) {
-    // the partial products are reduce-added: start from zero (same stream)
-    const size_t bytes = static_cast<size_t>(D) * cols * 4;
-    cudaError_t z = cudaMemsetAsync(dw, 0, bytes, stream);
-    if (z != cudaSuccess) return static_cast<int>(z) + 2;
-  }
   const int grid = p.n_units < num_sms ? p.n_units : num_sms;
   cudaError_t e = cudaFuncSetAttribute(relkl_wgrad_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, ALLOC);

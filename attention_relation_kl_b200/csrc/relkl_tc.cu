@@ -2005,32 +2005,50 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
             const int limr = rs ? lim[1] : lim[0];
             const int col0 = J * BN + wg * 32;
             const uint32_t gsm = gsm0 + (nt & 1) * L::G_BYTES;
-            // the logits are read in two 16-column halves, each turned into G and
-            // stored before the next is loaded (the second half releases the
-            // buffer): few values live at once, and the exps, which bound this
-            // kernel, leave time for the next tile's logit MMAs either way.  A
-            // full mask adds the transposed partners off the diagonal tile
-            // (4 exps per entry).
+            if constexpr (SYM) {
+              // full mask: 4 exps per entry off the diagonal tile, so the exps
+              // bound this mode; the logits are read in two 16-column halves
+              // (the second half releases the buffer), which keeps registers
+              // free for the partners' shuffles
 #pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {
-              float t[16], s[16];
-              tmem_ld16(ta + hf * 16, t);
-              tmem_ld16(ta + BN + hf * 16, s);
-              tmem_wait_ld();
-              if (hf == 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(S_EMPTY);
-              } else {
-                // the gradient MMAs of two tiles back have read this G buffer
-                ok = mbar_wait(G_EMPTY(nt & 1), ((nt >> 1) & 1) ^ 1, wc, W_SM_G_EMPTY);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
+              for (int hf = 0; hf < 2; ++hf) {
+                float t[16], s[16];
+                tmem_ld16(ta + hf * 16, t);
+                tmem_ld16(ta + BN + hf * 16, s);
+                tmem_wait_ld();
+                if (hf == 1) {
+                  tc_fence_before();
+                  __syncwarp();
+                  if (lane == 0) mbar_arrive(S_EMPTY);
+                } else {
+                  // the gradient MMAs of two tiles back have read this G buffer
+                  ok = mbar_wait(G_EMPTY(nt & 1), ((nt >> 1) & 1) ^ 1, wc, W_SM_G_EMPTY);
+                  ok = __all_sync(0xffffffffu, ok);
+                  if (!ok) break;
+                }
+                form_g_store<16>(t, s, btr, bsr, mr, col0 + hf * 16, limr, off, pc, hf * 16, p,
+                                 gsm, (wg & 1) * 4 + hf * 2, r);
               }
-              form_g_store<16>(t, s, btr, bsr, mr, col0 + hf * 16, limr, off, pc, hf * 16, p, gsm,
-                               (wg & 1) * 4 + hf * 2, r);
+              if (!ok) break;
+            } else {
+              // causal: read the whole slice of the tile at once and release the
+              // logit buffer at once, so the next tile's logit MMAs overlap this
+              // tile's exps (measured faster than two half loads despite the
+              // register pressure)
+              float t[32], s[32];
+              tmem_ld32(ta, t);
+              tmem_ld32(ta + BN, s);
+              tmem_wait_ld();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(S_EMPTY);
+              // the gradient MMAs of two tiles back have read this G buffer
+              ok = mbar_wait(G_EMPTY(nt & 1), ((nt >> 1) & 1) ^ 1, wc, W_SM_G_EMPTY);
+              ok = __all_sync(0xffffffffu, ok);
+              if (!ok) break;
+              form_g_store<32>(t, s, btr, bsr, mr, col0, limr, false, pc, 0, p, gsm,
+                               (wg & 1) * 4, r);
             }
-            if (!ok) break;
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(G_FULL(nt & 1));

@@ -351,7 +351,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="ext_h32_n32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--ref-prefix", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
@@ -495,13 +495,62 @@ def main():
     ms = max_over_ranks(ms, dev)
     peak_alloc = torch.cuda.max_memory_allocated(dev)
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: every step copies its
+    # inputs from pinned host memory and its kl rows and dX_s back.  Steps are
+    # pipelined over two buffer sets and three streams (host-to-device copies,
+    # compute, device-to-host copies), as a training loop would overlap the next
+    # batch's upload and the last batch's download with the current step; the
+    # context-parallel split, whose step holds collectives, runs them in order.
     e2e_ms = None
     h2d = sum(host[r][0].numel() * host[r][0].element_size() * 2 for r in rels)
-    host_dx = [torch.empty(d.shape, dtype=torch.float32, pin_memory=True) for d in dx_out]
-    host_kl = [torch.empty(k.shape, dtype=torch.float32, pin_memory=True) for k in kl_out]
-    d2h = sum(h.numel() * 4 for h in host_dx) + sum(h.numel() * 4 for h in host_kl)
-    if args.e2e_steps > 0:
+    d2h = sum(d.numel() * 4 for d in dx_out) + sum(k.numel() * 4 for k in kl_out)
+    if args.e2e_steps > 0 and split != "rows":
+        sets = []
+        for b in range(2):
+            bp = pairs if b == 0 else [(torch.empty_like(a), torch.empty_like(c)) for a, c in pairs]
+            bo = outs if b == 0 else [(torch.empty_like(k), torch.empty_like(st)) for k, st in outs]
+            bd = dxs if b == 0 else [torch.empty_like(d) for d in dxs]
+            hk = [torch.empty(k.shape, dtype=torch.float32, pin_memory=True) for k, _ in bo]
+            hd = [torch.empty(d.shape, dtype=torch.float32, pin_memory=True) for d in bd]
+            sets.append((bp, bo, bd, hk, hd))
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_cmp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s_in)
+        for i in range(args.e2e_steps):
+            b = i & 1
+            bp, bo, bd, hk, hd = sets[b]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[b])      # step i-2 has finished reading set b
+                for (gt, gs), r in zip(bp, rels):
+                    gt.copy_(host[r][0], non_blocking=True)
+                    gs.copy_(host[r][1], non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])        # step i-2's outputs have been copied out
+            rk.relkl_fwd_qkv(bp, w.causal, out=bo, ws=ws)
+            rk.relkl_bwd_qkv(bp, [o[1] for o in bo], None, w.causal, out=bd, ws=ws)
+            ev_cmp[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[b])
+                for h, (kl, _) in zip(hk, bo):
+                    h.copy_(kl, non_blocking=True)
+                for h, dv in zip(hd, bd):
+                    h.copy_(dv, non_blocking=True)
+                ev_out[b].record(s_out)
+        e1.record(s_out)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
+        del sets
+    elif args.e2e_steps > 0:
+        host_dx = [torch.empty(d.shape, dtype=torch.float32, pin_memory=True) for d in dx_out]
+        host_kl = [torch.empty(k.shape, dtype=torch.float32, pin_memory=True) for k in kl_out]
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -583,7 +632,9 @@ def main():
                                           "of the relkl_bwd_qkv call (dX zeroing included)"},
             "e2e": {"value": None if e2e_ms is None else total_fl / (e2e_ms * 1e-3) / 1e12,
                     "unit": "TFLOP/s", "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+                    "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps,
+                    "pipelined": split != "rows"},
             "gpu_launches": args.steps * (2 + len(w.relations)),
             "memory": {"peak_allocated_bytes": peak_alloc, "inputs_bytes": in_bytes,
                        "dx_bytes": out_dx_bytes, "row_stats_bytes": stats_bytes,
