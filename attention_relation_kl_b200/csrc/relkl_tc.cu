@@ -608,6 +608,7 @@ __host__ __device__ __forceinline__ int n_col_tiles_s(const TcParams& p, const U
 // (partner_column), and the entries take them from that lane by shuffles.
 struct PartnerCol {
   float bt, bs, mul;   // -lse_t log2 e, -lse_s log2 e, dkl * scale of one column
+  float ut, us;        // mul * 2^(bt - c_t), mul * 2^(bs - c_s): the column's share of the rescale
 };
 
 __device__ __forceinline__ PartnerCol partner_column(const Unit& U, const TcParams& p, int c) {
@@ -617,11 +618,41 @@ __device__ __forceinline__ PartnerCol partner_column(const Unit& U, const TcPara
   out.bt = -a.y * kLog2e;
   out.bs = -a.z * kLog2e;
   out.mul = (U.seg->dkl ? U.seg->dkl[U.row0 + cc] : 1.0f / static_cast<float>(U.len)) * p.scale;
+  out.ut = out.us = 0.f;
   return out;
 }
 
-// Adds the partners of the column pair held by lanes src, src + 1 to g; zt2 /
-// zs2 are the raw logit accumulators of the pair.
+// The partner of entry (i, j) is dkl_j (2^(zs l + bs_j) - 2^(zt l + bt_j)) with
+// l = scale log2 e.  Since 2^(zs l + bs_j) = 2^(zs l + bs_i) 2^(bs_j - bs_i), it
+// reuses the row side's exps: with a per-tile reference c (the first column's
+// bs), 2^(bs_j - bs_i) = 2^(c - bs_i) 2^(bs_j - c), a per-row times a
+// per-column factor, so H(i,j) = es (m_i + A_i^s u_j^s) - et (m_i + A_i^t u_j^t)
+// costs 2 exps per entry instead of 4.  Valid while every factor stays well
+// inside float range: |bs - c| <= 43 for the rows and columns of the tile (the
+// LSEs then differ by at most ~60, and a partner whose row-side exp
+// underflows is below 2^-80 of its column's largest term); a warp whose tile
+// leaves that range takes the 4-exp form.
+struct PartnerTile {
+  float at, as;   // 2^(c_t - bt_i), 2^(c_s - bs_i) of this thread's row
+  bool ok;        // the factored form holds for this warp's tile
+};
+
+__device__ __forceinline__ PartnerTile partner_tile(PartnerCol& pc, float bt_i, float bs_i) {
+  constexpr unsigned kAll = 0xffffffffu;
+  const float ct = __shfl_sync(kAll, pc.bt, 0), cs = __shfl_sync(kAll, pc.bs, 0);
+  const bool in = fabsf(ct - bt_i) <= 43.f && fabsf(cs - bs_i) <= 43.f &&
+                  fabsf(pc.bt - ct) <= 43.f && fabsf(pc.bs - cs) <= 43.f;
+  PartnerTile pt;
+  pt.ok = __all_sync(kAll, in);
+  pt.at = ex2_approx(ct - bt_i);
+  pt.as = ex2_approx(cs - bs_i);
+  pc.ut = pc.mul * ex2_approx(pc.bt - ct);
+  pc.us = pc.mul * ex2_approx(pc.bs - cs);
+  return pt;
+}
+
+// Adds the partners of the column pair held by lanes src, src + 1 to g (the
+// 4-exp form); zt2 / zs2 are the raw logit accumulators of the pair.
 __device__ __forceinline__ float2 sym_partner(const PartnerCol& pc, int src, float sl2, float2 zt2,
                                               float2 zs2, float2 g) {
   constexpr unsigned kAll = 0xffffffffu;
@@ -640,19 +671,31 @@ __device__ __forceinline__ float2 sym_partner(const PartnerCol& pc, int src, flo
 template <int NC>
 __device__ __forceinline__ void form_g_pack(const float (&t)[NC], const float (&s)[NC], float bt,
                                             float bs, float mul, int col0, int lim, bool off,
-                                            const PartnerCol& pc, int lane0, const TcParams& p,
-                                            uint32_t (&pk)[NC / 2]) {
+                                            const PartnerCol& pc, const PartnerTile& pt, int lane0,
+                                            const TcParams& p, uint32_t (&pk)[NC / 2]) {
+  constexpr unsigned kAll = 0xffffffffu;
   const float2 sl2v = make_float2(p.sl2, p.sl2), btv = make_float2(bt, bt),
                bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
-               m1 = make_float2(-1.f, -1.f);
+               m1 = make_float2(-1.f, -1.f), atv = make_float2(pt.at, pt.at),
+               asv = make_float2(pt.as, pt.as);
   const bool need_mask = col0 + NC - 1 > lim;
+  const bool fac = off && pt.ok;
 #pragma unroll
   for (int k = 0; k < NC; k += 2) {
     const float2 zt2 = make_float2(t[k], t[k + 1]), zs2 = make_float2(s[k], s[k + 1]);
     const float2 et = ex2_approx2(__ffma2_rn(zt2, sl2v, btv));
     const float2 es = ex2_approx2(__ffma2_rn(zs2, sl2v, bsv));
-    float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
-    if (off) g = sym_partner(pc, lane0 + k, p.sl2, zt2, zs2, g);
+    float2 g;
+    if (fac) {
+      const int src = lane0 + k;
+      const float2 ut = make_float2(__shfl_sync(kAll, pc.ut, src), __shfl_sync(kAll, pc.ut, src + 1));
+      const float2 us = make_float2(__shfl_sync(kAll, pc.us, src), __shfl_sync(kAll, pc.us, src + 1));
+      const float2 ft = __ffma2_rn(atv, ut, mulv), fs = __ffma2_rn(asv, us, mulv);
+      g = __ffma2_rn(es, fs, __fmul2_rn(__fmul2_rn(et, ft), m1));
+    } else {
+      g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
+      if (off) g = sym_partner(pc, lane0 + k, p.sl2, zt2, zs2, g);
+    }
     if (need_mask) {
       g.x = (col0 + k <= lim) ? g.x : 0.f;
       g.y = (col0 + k + 1 <= lim) ? g.y : 0.f;
@@ -1534,7 +1577,9 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
               // G plus its transposed partner (4 exps per entry); as in the causal
               // path the G buffer is awaited only once the entries are formed
               uint32_t pk[8];
-              form_g_pack<16>(t, s, btr, bsr, mr, col0, limr, off, pc, 0, p, pk);
+              PartnerTile pt{1.f, 1.f, false};
+              if (off) pt = partner_tile(pc, btr, bsr);
+              form_g_pack<16>(t, s, btr, bsr, mr, col0, limr, off, pc, pt, 0, p, pk);
               ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
               ok = __all_sync(0xffffffffu, ok);
               if (!ok) break;

@@ -342,6 +342,38 @@ def run_chain(args):
     return 0
 
 
+def run_wgrad(args):
+    """Time only the weight-gradient GEMM at the LLaMA2-7B layer shape (rows = 32768
+    tokens, D = 4096, cols = 32 heads x 128) on seeded bf16 operands: the inputs of
+    one relation's dW.  One JSON line."""
+    import attention_relation_kl_b200 as rk
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    rows, D, cols = 32768, 4096, 4096
+    gen = torch.Generator().manual_seed(43)
+    h = torch.randn(rows, D, generator=gen).to(torch.bfloat16).to(dev)
+    dx = torch.randn(rows, cols, generator=gen).to(torch.bfloat16).to(dev)
+    dw = torch.empty(D, cols, dtype=torch.float32, device=dev)
+    for _ in range(max(3, args.warmup)):
+        rk.relkl_weight_grad(h, dx, out=dw)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    steps = max(1, args.steps)
+    ev[0].record()
+    for _ in range(steps):
+        rk.relkl_weight_grad(h, dx, out=dw)
+    ev[1].record()
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / steps
+    peaks, src = load_peaks()
+    fl = 2.0 * rows * D * cols
+    print(json.dumps({"wgrad": f"rows={rows} D={D} cols={cols}", "ms": ms,
+                      "tflops": fl / (ms * 1e-3) / 1e12,
+                      "frac_bf16_burst": fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                      "peak_source": src}), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 
 def main():
@@ -360,6 +392,8 @@ def main():
     ap.add_argument("--chain", action="store_true",
                     help="time the chain rule to the Q/K/V weights (RoPE backward, weight "
                          "gradient GEMMs) at the LLaMA2-7B layer shape, N = 32768")
+    ap.add_argument("--wgrad", action="store_true",
+                    help="time only the weight-gradient GEMM at the LLaMA2-7B layer shape")
     ap.add_argument("--split", default="replicas", choices=["replicas", "units", "rows"],
                     help="how N ranks share work: 'replicas' (default) runs one replica of the "
                          "workload per rank (weak scaling); 'units' splits one problem's heads "
@@ -375,6 +409,8 @@ def main():
         return run_sweep(args)
     if args.chain:
         return run_chain(args)
+    if args.wgrad:
+        return run_wgrad(args)
 
     import torch.distributed as dist
     import attention_relation_kl_b200 as rk
