@@ -179,6 +179,10 @@ relkl_bwd_simt_kernel(const __grid_constant__ SimtParams p) {
     lse_t = st4.y;
     lse_s = st4.z;
     mul = (S.dkl ? S.dkl[U.row0 + row] : 1.0f / static_cast<float>(U.L)) * sc;
+    // a row with one allowed entry has R_t = R_s = 1 there: its gradient is
+    // exactly zero (left to the exps, float32 rounding of logits and LSEs of
+    // size ~|z| would leave ~|z| 2^-24 of it, times the row's upstream weight)
+    if (p.causal ? row == 0 : U.L == 1) mul = 0.f;
   }
   // dX_I accumulator: this thread owns columns cg, cg+8, ... of row rr
   constexpr int MAXC = 128 / 8;

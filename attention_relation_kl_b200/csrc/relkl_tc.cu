@@ -1052,6 +1052,7 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
           mul = up * p.scale;   // the logit scale of dX_s is folded into G
         }
         const int lim = !rvalid ? -1 : (p.causal ? min(row, L - 1) : L - 1);
+        if (lim == 0) mul = 0.f;   // one allowed entry: R_t = R_s = 1, the gradient is 0
         const int nT = n_col_tiles64(p, U, I);
         const float2 sl2v = make_float2(sl2, sl2), btv = make_float2(bt, bt),
                      bsv = make_float2(bs, bs), mulv = make_float2(mul, mul),
@@ -1126,8 +1127,11 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
 // tiles that only R1 reaches under the causal mask run alone.  Two warps
 // issue MMAs: one the logits of the next tile, one the gradient products of
 // the tile whose G was just stored.
-//   TMEM: Z_t/Z_s 0..127 (one buffer: the row warps read all of it at once
-//         and release it), dX_R0 128..255, dX_R1 256..383, P^T 2 x 64 at 384.
+//   TMEM: Z_t 0..63, Z_s 64..127 (one buffer; under the causal mask the row
+//         warps read Z_t, release it and form the teacher's exps while Z_s is
+//         computed, and the next tile's Z_t is computed while they read Z_s;
+//         the full mask reads and releases both at once), dX_R0 128..255,
+//         dX_R1 256..383, P^T 2 x 64 at 384.
 //   smem: X_t, X_s of R0 and R1 (4 x 32 KB); teacher and student column
 //         rings 2 x 16 KB each; G 16 KB; epilogue staging 4 x 4 KB.
 // A work item is the pair sequence k = npb-1-m followed by k = m (npb row-block
@@ -1151,8 +1155,9 @@ struct BwdPairSmem {
   static constexpr int STG_BYTES = 32 * 32 * 4;
   static constexpr int BARS = STG + 4 * STG_BYTES;
   // full_I, empty_I, fullT[2], emptyT[2], fullS[2], emptyS[2], s_full, s_empty,
-  // g_full, g_empty, p_full[2], p_empty[2], dxi_full, dxi_empty, drain x 2
-  static constexpr int NBAR = 22;
+  // g_full, g_empty, p_full[2], p_empty[2], dxi_full, dxi_empty, drain x 2,
+  // t_full, t_empty
+  static constexpr int NBAR = 24;
   static constexpr int MISC = BARS + NBAR * 8;
   static constexpr int BYTES = MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
@@ -1197,6 +1202,9 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
   auto P_FULL = [&](int b) { return BAR(14 + b); };
   auto P_EMPTY = [&](int b) { return BAR(16 + b); };
   const uint32_t DXI_FULL = BAR(18), DXI_EMPTY = BAR(19), DRAIN_L = BAR(20), DRAIN_G = BAR(21);
+  // causal mask: T_FULL / T_EMPTY guard Z_t, S_FULL / S_EMPTY Z_s; full mask:
+  // S_FULL / S_EMPTY guard both
+  const uint32_t T_FULL = BAR(22), T_EMPTY = BAR(23);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
 
@@ -1220,6 +1228,8 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
     }
     mbar_init(S_FULL, 1);
     mbar_init(S_EMPTY, 16);
+    mbar_init(T_FULL, 1);
+    mbar_init(T_EMPTY, 16);
     mbar_init(G_FULL, 16);
     mbar_init(G_EMPTY, 1);
     mbar_init(DXI_FULL, 1);
@@ -1346,9 +1356,12 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
             const bool first_p = rs == 0 || J >= nT0;
             const bool last_p = rs == 1 || !has1;
             if (is_logit) {
-              // Z_t, Z_s of tile (R, J) into the logit buffer
+              // Z_t, Z_s of tile (R, J) into the logit buffer; under the causal mask
+              // Z_t as soon as the row warps have read the previous Z_t, Z_s once
+              // they have read the previous Z_s
               if (!(ok = mbar_wait_warp(FULL_T(tt), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
-              if (!(ok = mbar_wait_warp(S_EMPTY, (nt & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
+              if (!(ok = mbar_wait_warp(SYM ? S_EMPTY : T_EMPTY, (nt & 1) ^ 1, wc, W_MMA_S_EMPTY)))
+                break;
               tc_fence_after();
               const uint32_t xtj = dXtJ_k0 + tt * J_STEP, xsj = dXsJ_k0 + ts * J_STEP;
               // K steps: 32 B within a 128 B row, then the next 64-column box
@@ -1359,7 +1372,9 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
                                  IDESC_S, k > 0 ? 1u : 0u);
               issued = true;
               if (last_p) umma_commit_lead(lead, EMPTY_T(tt));
+              if (!SYM) umma_commit_lead(lead, T_FULL);
               if (!(ok = mbar_wait_warp(FULL_S(ts), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+              if (!SYM && !(ok = mbar_wait_warp(S_EMPTY, (nt & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
               tc_fence_after();
 #pragma unroll
               for (int k = 0; k < D / 16; ++k)
@@ -1542,6 +1557,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
             mul[rs] = up * p.scale;   // the logit scale of dX_s is folded into G
           }
           lim[rs] = !rvalid ? -1 : (p.causal ? min(row, L - 1) : L - 1);
+          if (lim[rs] == 0) mul[rs] = 0.f;   // one allowed entry: R_t = R_s = 1, the gradient is 0
         }
         const float2 sl2v = make_float2(sl2, sl2), m1 = make_float2(-1.f, -1.f);
         for (int J = 0; ok && J < nT; ++J) {
@@ -1554,24 +1570,43 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
             const bool off = SYM && J < 2 * (R0 + rs);
             PartnerCol pc{0.f, 0.f, 0.f};
             if (off) pc = partner_column(U, p, J * BN64 + wg * 16 + (lane & 15));
-            ok = mbar_wait(S_FULL, nt & 1, wc, W_SM_S_FULL);
+            ok = mbar_wait(SYM ? S_FULL : T_FULL, nt & 1, wc, W_SM_S_FULL);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
             const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + T_S + wg * 16;
             float t[16], s[16];
             tmem_ld16(ta, t);
-            tmem_ld16(ta + 64, s);
+            if constexpr (SYM) tmem_ld16(ta + 64, s);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(S_EMPTY);
+            if (lane == 0) mbar_arrive(SYM ? S_EMPTY : T_EMPTY);
             const float btr = rs ? bt[1] : bt[0], bsr = rs ? bs[1] : bs[0];
             const float mr = rs ? mul[1] : mul[0];
             const int limr = rs ? lim[1] : lim[0];
             const float2 btv = make_float2(btr, btr), bsv = make_float2(bsr, bsr),
                          mulv = make_float2(mr, mr);
             const int col0 = J * BN64 + wg * 16;
+            if constexpr (!SYM) {
+              // the teacher's exps while Z_s is still being computed (t then holds
+              // e_t), then Z_s
+#pragma unroll
+              for (int k = 0; k < 16; k += 2) {
+                const float2 et = ex2_approx2(__ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv));
+                t[k] = et.x;
+                t[k + 1] = et.y;
+              }
+              ok = mbar_wait(S_FULL, nt & 1, wc, W_SM_S_FULL);
+              ok = __all_sync(0xffffffffu, ok);
+              if (!ok) break;
+              tc_fence_after();
+              tmem_ld16(ta + 64, s);
+              tmem_wait_ld();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(S_EMPTY);
+            }
             if constexpr (SYM) {
               // full mask: tiles of the diagonal block carry G itself, the others
               // G plus its transposed partner (4 exps per entry); as in the causal
@@ -1594,10 +1629,8 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
             uint32_t pk[8];
 #pragma unroll
             for (int k = 0; k < 16; k += 2) {
-              const float2 at = __ffma2_rn(make_float2(t[k], t[k + 1]), sl2v, btv);
-              const float2 as = __ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv);
-              const float2 et = ex2_approx2(at), es = ex2_approx2(as);
-              float2 g = __fmul2_rn(__ffma2_rn(et, m1, es), mulv);
+              const float2 es = ex2_approx2(__ffma2_rn(make_float2(s[k], s[k + 1]), sl2v, bsv));
+              float2 g = __fmul2_rn(__ffma2_rn(make_float2(t[k], t[k + 1]), m1, es), mulv);
               if (need_mask) {
                 g.x = (col0 + k <= limr) ? g.x : 0.f;
                 g.y = (col0 + k + 1 <= limr) ? g.y : 0.f;
@@ -2028,6 +2061,7 @@ relkl_bwd_pair64_kernel(const __grid_constant__ TcParams p) {
             mul[rs] = up * p.scale;   // the logit scale of dX_s is folded into G
           }
           lim[rs] = !rvalid ? -1 : (p.causal ? min(row, Lu - 1) : Lu - 1);
+          if (lim[rs] == 0) mul[rs] = 0.f;   // one allowed entry: R_t = R_s = 1, the gradient is 0
         }
         const float2 sl2v = make_float2(sl2, sl2), m1 = make_float2(-1.f, -1.f);
         for (int J = 0; ok && J < nT; ++J) {

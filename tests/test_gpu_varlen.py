@@ -65,6 +65,10 @@ def test_packed_sequences(lens, d, dtype, causal):
         for a, b in zip(cu[:-1], cu[1:]) if b > a)
     assert_dx(to_np(dx), ref_dx, tol)
     assert np.all(to_np(dx)[:, :, end:] == 0)
+    # a sequence of one token: its only row has R_t = R_s = 1, so its gradient is exactly 0
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b - a == 1:
+            assert np.all(to_np(dx)[:, :, a] == 0)
 
 
 def test_packed_sequences_fused_qkv_and_upstream_gradient():
