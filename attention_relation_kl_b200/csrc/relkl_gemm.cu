@@ -23,11 +23,7 @@
 //     stored by TMA (tiles past the matrix edge are clipped by TMA).
 // Tiles are taken M-fastest, so the CTAs that run together share the B panels
 // of a few column blocks and walk K in step, which keeps the K slices of both
-// operands in L2.  When the tiles leave a last wave that fills at most half of
-// the CTAs, those tiles are split into two 128 x 128 halves, so the last wave
-// takes half as long (at the LLaMA2-7B shape: 512 tiles on 148 CTAs, three
-// full waves and 68 tiles, run as 136 halves).  Every wait is bounded like the
-// relation-KL kernels'.
+// operands in L2.  Every wait is bounded like the relation-KL kernels'.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -66,25 +62,18 @@ struct GemmParams {
   CUtensorMap tm_c;   // dW [D, cols] f32: dims {cols, D}, box {32, 32}, 128B swizzle
   int m_tiles, n_tiles, k_chunks;
   int D, cols;        // the output's extent: boxes that start past it are not stored
-  int n_big;          // units [0, n_big) are 128 x 256 tiles, the rest 128 x 128 halves
-  int n_units;
+  int n_units;        // m_tiles * n_tiles output tiles
   DevStatus* status;
   unsigned long long timeout_ns;
 };
 
-// Work unit -> (M tile, first column, whether it is a full 256-column tile):
-// M-fastest tiles over all of K; units past n_big are the two column halves
-// of the tiles that remain.
-__device__ __forceinline__ void gemm_unit(const GemmParams& p, int unit, int& mt, int& n0,
-                                          bool& wide) {
-  int tile = unit, half = 0;
-  wide = unit < p.n_big;
-  if (!wide) {
-    tile = p.n_big + ((unit - p.n_big) >> 1);
-    half = (unit - p.n_big) & 1;
-  }
-  mt = tile % p.m_tiles;
-  n0 = (tile / p.m_tiles) * gemm::BN + half * (gemm::BN / 2);
+// Work unit -> (M tile, N tile, chunk range [k0, k1)): M-fastest tiles, all of K.
+__device__ __forceinline__ void gemm_unit(const GemmParams& p, int unit, int& mt, int& nt,
+                                          int& k0, int& k1) {
+  mt = unit % p.m_tiles;
+  nt = unit / p.m_tiles;
+  k0 = 0;
+  k1 = p.k_chunks;
 }
 
 __global__ void __launch_bounds__(gemm::THREADS, 1)
@@ -138,20 +127,19 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
       uint32_t arms[STAGES] = {0, 0, 0, 0};
       bool ok = true;
       for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
-        int mt, n0;
-        bool wide;
-        gemm_unit(p, unit, mt, n0, wide);
-        const int nb = wide ? BN / 64 : BN / 128;   // B boxes per stage
-        for (int kc = 0; kc < p.k_chunks; ++kc, ++it) {
+        int mt, nt, k0, k1;
+        gemm_unit(p, unit, mt, nt, k0, k1);
+        for (int kc = k0; kc < k1; ++kc, ++it) {
           const int s = it % STAGES;
           if (!(ok = mbar_wait(EMPTY(s), ((it / STAGES) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
           const uint32_t a = base + s * STAGE_BYTES, b = a + A_BYTES;
-          mbar_arrive_expect_tx(FULL(s), A_BYTES + nb * BOX);
+          mbar_arrive_expect_tx(FULL(s), STAGE_BYTES);
 #pragma unroll
           for (int i = 0; i < BM / 64; ++i)
             tma_load_2d(a + i * BOX, &p.tm_a, FULL(s), mt * BM + i * 64, kc * BK);
-          for (int i = 0; i < nb; ++i)
-            tma_load_2d(b + i * BOX, &p.tm_b, FULL(s), n0 + i * 64, kc * BK);
+#pragma unroll
+          for (int i = 0; i < BN / 64; ++i)
+            tma_load_2d(b + i * BOX, &p.tm_b, FULL(s), nt * BN + i * 64, kc * BK);
           ++arms[s];
         }
       }
@@ -165,7 +153,6 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
     // A = H_s^T and B = dX_pre are MN-major: 64-element blocks of M (N) are
     // one box apart (LBO), K steps 16 rows = 2 KB
     constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 1, 1);
-    constexpr uint32_t IDESC_HALF = idesc_bf16_f32(BM, BN / 2, 1, 1);
     const uint32_t HI = sw128_desc_hi(1024);
     const uint32_t a0 = sw128_desc_lo(base, BOX);
     const uint32_t b0 = sw128_desc_lo(base + A_BYTES, BOX);
@@ -173,22 +160,20 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
     uint32_t it = 0, nacc = 0;
     bool ok = true, issued = false;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x, ++nacc) {
-      int mt, n0;
-      bool wide;
-      gemm_unit(p, unit, mt, n0, wide);
-      const uint32_t idesc = wide ? IDESC : IDESC_HALF;
+      int mt, nt, k0, k1;
+      gemm_unit(p, unit, mt, nt, k0, k1);
       const int ab = nacc & 1;
       if (!(ok = mbar_wait_warp(ACC_EMPTY(ab), ((nacc >> 1) & 1) ^ 1, wc, W_MMA_P_EMPTY))) break;
       tc_fence_after();
       const uint32_t acc = tmem + ab * BN;
-      for (int kc = 0; kc < p.k_chunks; ++kc, ++it) {
+      for (int kc = k0; kc < k1; ++kc, ++it) {
         const int s = it % STAGES;
         if (!(ok = mbar_wait_warp(FULL(s), (it / STAGES) & 1, wc, W_MMA_FULL_J))) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
           umma_bf16_w_lead(lead, acc, a0 + s * STAGE_STEP + k * 128, HI,
-                           b0 + s * STAGE_STEP + k * 128, HI, idesc, (kc > 0 || k > 0) ? 1u : 0u);
+                           b0 + s * STAGE_STEP + k * 128, HI, IDESC, (kc > k0 || k > 0) ? 1u : 0u);
         issued = true;
         umma_commit_lead(lead, EMPTY(s));
       }
@@ -208,21 +193,19 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
     uint32_t nacc = 0, nstg = 0;
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x, ++nacc) {
-      int mt, n0;
-      bool wide;
-      gemm_unit(p, unit, mt, n0, wide);
-      const int nc = wide ? BN / 32 : BN / 64;   // 32-column boxes of this unit
+      int mt, nt, k0, k1;
+      gemm_unit(p, unit, mt, nt, k0, k1);
       const int ab = nacc & 1;
       ok = mbar_wait(ACC_FULL(ab), (nacc >> 1) & 1, wc, W_EPI_P_FULL);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < nc; ++c) {
+      for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_ld32(tmem + lane_addr + ab * BN + c * 32, v);
         tmem_wait_ld();
-        if (c == nc - 1) {
+        if (c == BN / 32 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(ACC_EMPTY(ab));
@@ -239,8 +222,8 @@ relkl_wgrad_kernel(const __grid_constant__ GemmParams p) {
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (n0 + c * 32 < p.cols && mt * BM + q * 32 < p.D)
-            tma_store_2d(&p.tm_c, buf, n0 + c * 32, mt * BM + q * 32);
+          if (nt * BN + c * 32 < p.cols && mt * BM + q * 32 < p.D)
+            tma_store_2d(&p.tm_c, buf, nt * BN + c * 32, mt * BM + q * 32);
           bulk_commit();
         }
         ++nstg;
@@ -300,15 +283,10 @@ int launch_wgrad(EncodeTiledFnG encode, long long rows, int D, int cols, const v
   p.k_chunks = static_cast<int>((rows + BK - 1) / BK);
   p.D = D;
   p.cols = cols;
-  const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  // a last wave that would fill at most half of the CTAs runs as column halves
-  const int rem = tiles % grid;
-  const bool split = rem > 0 && 2 * rem <= grid && tiles > grid;
-  p.n_big = split ? tiles - rem : tiles;
-  p.n_units = split ? tiles + rem : tiles;
+  p.n_units = p.m_tiles * p.n_tiles;
   p.status = status;
   p.timeout_ns = timeout_ns;
+  const int grid = p.n_units < num_sms ? p.n_units : num_sms;
   cudaError_t e = cudaFuncSetAttribute(relkl_wgrad_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, ALLOC);
   if (e == cudaSuccess) {

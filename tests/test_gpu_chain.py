@@ -57,9 +57,9 @@ def test_rope_bwd_without_rotation_is_an_exact_transpose_and_cast():
     assert torch.equal(out16.cpu(), want.to(torch.bfloat16))   # round to nearest even
 
 
-# (1000, 1280, 3968) and (1000, 1280, 3904): 160 tiles on 148 SMs, so the last 12 tiles
-# run as column halves; in the last column block the second half lies wholly (3968) or
-# partly (3904) past the matrix edge
+# (1000, 1280, 3968) and (1000, 1280, 3904): the last 256-column block reaches past the
+# matrix edge by half (3968: its last four 32-column boxes are not stored) or more (3904),
+# and the 1000 token rows end inside a 64-row K chunk
 @pytest.mark.parametrize("rows,D,cols", [(600, 192, 256), (32768, 256, 128), (40, 8, 8),
                                          (1000, 1280, 3968), (1000, 1280, 3904)])
 def test_weight_grad_matches_float64(rows, D, cols):
