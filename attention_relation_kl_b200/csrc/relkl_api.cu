@@ -23,6 +23,8 @@ cudaError_t tc_launch_bwd(const TcParams& p, int d, int grid, cudaStream_t strea
 cudaError_t simt_launch_fwd(const SimtParams& p, cudaStream_t stream);
 cudaError_t simt_launch_bwd(const SimtParams& p, cudaStream_t stream);
 cudaError_t launch_zero(float* ptr, int64_t n, int num_sms, cudaStream_t stream);
+cudaError_t launch_cast_bf16(const float* src, void* dst, int64_t n, int num_sms,
+                             cudaStream_t stream);
 int schedule_check(const TcParams& p0, int d, bool bwd, int n_parts, const int* const* lens,
                    const int* const* offs, char* why, size_t why_len);
 cudaError_t launch_rope_bwd(const float* dx, void* out, int B, int H, int N, int d, bool bf16_out,
@@ -468,7 +470,7 @@ relkl_status bwd_impl(int32_t n_rel, const relkl_desc* descs, const void* const*
     build_simt(n_rel, descs, x_t, x_s, &sp, part, n_parts);
     set_seg_outputs(&sp, n_rel, descs, nullptr, nullptr, stats, dkl, dx_s);
   }
-  // dX_s is accumulated with atomics: clear it first (same stream)
+  // dX_s is accumulated by reduce-adds in L2: clear it first (same stream)
   for (int r = 0; r < n_rel; ++r) {
     if (!n_units(descs[r])) continue;
     // the whole [B, H, N, d] tensor (packed sequences: B = 1, every token)
@@ -625,6 +627,22 @@ relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const fl
   cudaError_t e = launch_rope_bwd(dx_post, dx_pre, B, H, N, d, out_dtype == RELKL_BF16, rope->base,
                                   rope->pos_scale, rope->pos_offset, rope->apply,
                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
+}
+
+relkl_status relkl_cast_bf16(const float* src, void* dst, int64_t n, void* stream) {
+  NvtxRange nvtx_range("relkl_cast_bf16");
+  if (n < 0) return RELKL_ERR_INVALID;
+  if (n == 0) return RELKL_OK;
+  if (!src || !dst || !aligned(src, 4) || !aligned(dst, 2)) return RELKL_ERR_INVALID;
+  // the two ranges may not overlap
+  const char* a = reinterpret_cast<const char*>(src);
+  const char* b = static_cast<const char*>(dst);
+  if (a < b + 2 * n && b < a + 4 * n) return RELKL_ERR_INVALID;
+  relkl_status s;
+  DevInfo dev;
+  if ((s = device_info(&dev)) != RELKL_OK) return s;
+  cudaError_t e = launch_cast_bf16(src, dst, n, dev.sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? RELKL_OK : cuda_fail(e);
 }
 

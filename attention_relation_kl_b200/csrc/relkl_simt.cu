@@ -291,4 +291,52 @@ cudaError_t launch_zero(float* ptr, int64_t n, int num_sms, cudaStream_t stream)
   return cudaGetLastError();
 }
 
+// ------------------------------------------------ bf16 copy of dX_s
+// Round to nearest, ties to even (cvt.rn), eight elements per thread step:
+// two 16-byte loads, one 16-byte store.  HBM-bound: 6 bytes per element.
+__global__ void relkl_cast_bf16_kernel(const float4* __restrict__ src, uint4* __restrict__ dst,
+                                       int64_t n8) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 a = src[2 * i], b = src[2 * i + 1];
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+    const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+    uint4 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&p0);
+    o.y = *reinterpret_cast<const uint32_t*>(&p1);
+    o.z = *reinterpret_cast<const uint32_t*>(&p2);
+    o.w = *reinterpret_cast<const uint32_t*>(&p3);
+    dst[i] = o;
+  }
+}
+
+// Element by element: the ragged tail, or arrays not 16-byte aligned.
+__global__ void relkl_cast_bf16_scalar_kernel(const float* __restrict__ src,
+                                              __nv_bfloat16* __restrict__ dst, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+cudaError_t launch_cast_bf16(const float* src, void* dst, int64_t n, int num_sms,
+                             cudaStream_t stream) {
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  auto blocks_for = [&](int64_t work) {
+    const int64_t b = (work + 255) / 256;
+    return static_cast<int>(b < cap ? b : cap);
+  };
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(dst);
+  const bool vec = (reinterpret_cast<uintptr_t>(src) % 16 == 0) &&
+                   (reinterpret_cast<uintptr_t>(dst) % 16 == 0);
+  const int64_t n8 = vec ? n / 8 : 0;
+  if (n8 > 0)
+    relkl_cast_bf16_kernel<<<blocks_for(n8), 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(src), reinterpret_cast<uint4*>(out), n8);
+  const int64_t rest = n - n8 * 8;
+  if (rest > 0)
+    relkl_cast_bf16_scalar_kernel<<<blocks_for(rest), 256, 0, stream>>>(src + n8 * 8, out + n8 * 8,
+                                                                        rest);
+  return cudaGetLastError();
+}
+
 }  // namespace relkl

@@ -22,7 +22,8 @@ from ._abi import check, relkl_desc
 __all__ = ["relkl_fwd", "relkl_bwd", "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_workspace_bytes",
            "relkl_workspace_init", "relkl_get_device_error", "relkl_set_wait_timeout_ns",
            "relkl_path_for", "workspace", "make_desc", "relation_kl", "RelationKL",
-           "relkl_fwd_noalloc", "relkl_rope_bwd", "relkl_weight_grad", "student_weight_grads"]
+           "relkl_fwd_noalloc", "relkl_rope_bwd", "relkl_weight_grad", "student_weight_grads",
+           "relkl_cast_bf16"]
 
 _DTYPES = {torch.bfloat16: _abi.RELKL_BF16, torch.float32: _abi.RELKL_FP32}
 
@@ -204,10 +205,14 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
                   ws: Optional[torch.Tensor] = None, stream=None,
                   lengths: Optional[torch.Tensor] = None, part=None,
                   cu_seqlens: Optional[torch.Tensor] = None,
-                  max_seqlen: int = 0) -> List[torch.Tensor]:
+                  max_seqlen: int = 0, dx_dtype: torch.dtype = torch.float32) -> List[torch.Tensor]:
     """Backward over 1..3 relations in one launch.  Returns dX_s per relation (float32).
     ``part``: (index, count) to return only that part's rows' contribution to
-    dX_s (relkl_bwd_qkv_part); ``stats`` must then hold every row."""
+    dX_s (relkl_bwd_qkv_part); ``stats`` must then hold every row.
+    ``dx_dtype=torch.bfloat16`` returns bf16 copies instead (relkl_cast_bf16 of
+    the float32 result, which is then ``out`` or a temporary)."""
+    if dx_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("dx_dtype must be torch.float32 or torch.bfloat16")
     p_idx, n_parts = _part(part)
     n = len(pairs)
     if not 1 <= n <= 3 or len(stats) != n:
@@ -241,7 +246,27 @@ def relkl_bwd_qkv(pairs: Sequence[Tuple[torch.Tensor, torch.Tensor]], stats: Seq
         else:
             code = _abi.lib().relkl_bwd_qkv_part(*args, p_idx, n_parts, *tail)
     check(code, "relkl_bwd_qkv")
+    if dx_dtype == torch.bfloat16:
+        return [relkl_cast_bf16(dx, stream=stream) for dx in dxs]
     return dxs
+
+
+def relkl_cast_bf16(src: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """bf16 copy of a float32 tensor (round to nearest, ties to even)."""
+    _cuda(src, "src")
+    if src.dtype != torch.float32 or not src.is_contiguous():
+        raise ValueError("src must be a contiguous float32 tensor")
+    if out is None:
+        out = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device)
+    if (out.dtype != torch.bfloat16 or not out.is_contiguous() or out.device != src.device
+            or out.numel() != src.numel()):
+        raise ValueError("out must be a contiguous bfloat16 tensor of src's size on its device")
+    with torch.cuda.device(src.device):
+        code = _abi.lib().relkl_cast_bf16(_ptr(src), _ptr(out), src.numel(),
+                                          _stream(src.device, stream))
+    check(code, "relkl_cast_bf16")
+    return out
 
 
 def relkl_fwd(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True, scale: float = 0.0, *,
@@ -262,11 +287,14 @@ def relkl_bwd(x_t: torch.Tensor, x_s: torch.Tensor, stats: torch.Tensor,
               dkl: Optional[torch.Tensor] = None, causal: bool = True, scale: float = 0.0, *,
               dx_s: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
               stream=None, lengths: Optional[torch.Tensor] = None,
-              cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: int = 0) -> torch.Tensor:
-    """dL/dX_s (float32) with L = sum_i dkl_i kl_i (dkl=None: 1/N per row, 1/L_b with lengths)."""
+              cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: int = 0,
+              dx_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    """dL/dX_s (float32, or a bf16 copy with dx_dtype=torch.bfloat16) with
+    L = sum_i dkl_i kl_i (dkl=None: 1/N per row, 1/L_b with lengths)."""
     return relkl_bwd_qkv([(x_t, x_s)], [stats], None if dkl is None else [dkl], causal, scale,
                          out=None if dx_s is None else [dx_s], ws=ws, stream=stream,
-                         lengths=lengths, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)[0]
+                         lengths=lengths, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen,
+                         dx_dtype=dx_dtype)[0]
 
 
 def relkl_fwd_noalloc(x_t: torch.Tensor, x_s: torch.Tensor, causal: bool = True,

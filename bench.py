@@ -321,6 +321,19 @@ def run_chain(args):
         bwd_ms += ev[0].elapsed_time(ev[1]) / steps
         rope_ms += ev[1].elapsed_time(ev[2]) / steps
         gemm_ms += ev[2].elapsed_time(ev[3]) / steps
+    # the optional bf16 copy of dX_s (relkl_cast_bf16), for the three relations
+    dx16 = [torch.empty(dx.shape, dtype=torch.bfloat16, device=dev) for dx in dxs]
+    for _ in range(3):
+        for dx, o in zip(dxs, dx16):
+            rk.relkl_cast_bf16(dx, out=o)
+    torch.cuda.synchronize()
+    ev[0].record()
+    for _ in range(steps):
+        for dx, o in zip(dxs, dx16):
+            rk.relkl_cast_bf16(dx, out=o)
+    ev[1].record()
+    torch.cuda.synchronize()
+    cast_ms = ev[0].elapsed_time(ev[1]) / steps
     peaks, src = load_peaks()
     elems = sum(dx.numel() for dx in dxs)
     rope_bytes = elems * (4 + 2)
@@ -335,6 +348,8 @@ def run_chain(args):
         "weight_grad_ms": gemm_ms, "weight_grad_tflops": gemm_fl / (gemm_ms * 1e-3) / 1e12,
         "weight_grad_frac_bf16": gemm_fl / (gemm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "weight_grad_flops": gemm_fl,
+        "dx_cast_bf16_ms": cast_ms, "dx_cast_bf16_gbs": rope_bytes / (cast_ms * 1e-3) / 1e9,
+        "dx_cast_bf16_frac_hbm": rope_bytes / (cast_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "relation_bwd_ms": bwd_ms,
         "chain_share_of_bwd": (rope_ms + gemm_ms) / bwd_ms,
         "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"], "source": src},

@@ -288,6 +288,21 @@ relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const fl
                             const relkl_rope* rope, int32_t out_dtype, void* dx_pre,
                             void* stream);
 
+/* bfloat16 copy of a float32 array, for a caller that keeps dX_s in bf16:
+ *
+ *   dst[i] = src[i] rounded to the nearest bf16, ties to even
+ *
+ * (overflow rounds to infinity, NaN stays NaN).  The pages fix only that dX_s
+ * is accumulated in float32 (the verdict page's Phase 2 streams it to the
+ * student's Q/K/V); the copy is a storage convenience and runs as its own
+ * HBM-bound pass, since a row of dX_s is complete only after every CTA that
+ * adds into it has done so.  Issue it on the stream of the relkl_bwd call.
+ *   src : float [n] (relkl_bwd's dx_s), in, 4-byte aligned.
+ *   dst : bf16 [n], out, 2-byte aligned; must not overlap src.
+ * n == 0 is a no-op (pointers unused).  RELKL_ERR_INVALID for n < 0, null or
+ * misaligned pointers, or overlapping ranges.  Asynchronous on `stream`.     */
+relkl_status relkl_cast_bf16(const float* src, void* dst, int64_t n, void* stream);
+
 /* Weight gradient over the token rows:
  *
  *   dw[D, cols] = h[rows, D]^T dx_pre[rows, cols]

@@ -7,7 +7,9 @@ never calls it.
 
 ``oracle.dense``  the definition (dense float64, optionally over row slabs).
 ``oracle.tiled``  tiled linear-memory restatements, checked against ``dense``.
+``oracle.chain``  the chain rule to the student's projection weights.
+``oracle.cast``   bfloat16 rounding (ties to even) of the float32 gradient.
 """
-from . import dense, tiled  # noqa: F401
+from . import cast, dense, tiled  # noqa: F401
 
-__all__ = ["dense", "tiled"]
+__all__ = ["cast", "dense", "tiled"]
