@@ -1132,12 +1132,16 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
 //         computed, and the next tile's Z_t is computed while they read Z_s;
 //         the full mask reads and releases both at once), dX_R0 128..255,
 //         dX_R1 256..383, P^T 2 x 64 at 384.
-//   smem: X_t, X_s of R0 and R1 (4 x 32 KB); teacher and student column
-//         rings 2 x 16 KB each; G 16 KB; epilogue staging 4 x 4 KB.
+//   smem: X_t, X_s of R0 and R1 (4 x 32 KB); one ring of 16 KB slots for the
+//         teacher and student column tiles; G; epilogue staging 4 x 4 KB.
+//         Causal mask: 3 slots and G 2 x 16 KB (the row warps store tile t's
+//         G while the gradient MMAs of tile t-1 read the other buffer); full
+//         mask: 4 slots and G 16 KB.
 // A work item is the pair sequence k = npb-1-m followed by k = m (npb row-block
 // pairs per unit), which evens out the causal triangle across items.  With
 // few row blocks the items are too coarse to balance 148 SMs, so sequences of
 // at most 32 row blocks use relkl_bwd_tc64_kernel instead.
+template <bool SYM>
 struct BwdPairSmem {
   static constexpr int TILE_I = BM * 128 * 2;        // 128 rows: boxes of 128 x 64 (16 KB)
   static constexpr int BOX_I = BM * 128;
@@ -1147,22 +1151,33 @@ struct BwdPairSmem {
   static constexpr int XS_R0 = TILE_I;
   static constexpr int XT_R1 = 2 * TILE_I;
   static constexpr int XS_R1 = 3 * TILE_I;
-  static constexpr int XT_J = 4 * TILE_I;            // 2 stages
-  static constexpr int XS_J = XT_J + 2 * TILE_J;     // 2 stages
-  static constexpr int G = XS_J + 2 * TILE_J;        // 128 x 64 bf16
+  // column tiles: one ring of 16 KB slots shared by the teacher and student
+  // tiles, taken in the order X_t[J], X_s[J], X_t[J+1], ... (the teacher tile
+  // leaves after its logit MMAs, the student tile only after the gradient MMAs
+  // of its last row block).  Causal mask: three slots and two G buffers; full
+  // mask (more row-warp work per tile, where the second G buffer measured
+  // slower than a fourth slot): four slots and one G buffer.
+  static constexpr int NSLOT = SYM ? 4 : 3;
+  static constexpr int NG = SYM ? 1 : 2;
+  static constexpr int RING = 4 * TILE_I;
+  static constexpr int G = RING + NSLOT * TILE_J;    // NG x (128 x 64 bf16)
   static constexpr int G_BYTES = BM * 64 * 2;
-  static constexpr int STG = G + G_BYTES;            // 4 warps x one 32 x 32 f32 box
+  static constexpr int STG = G + NG * G_BYTES;       // 4 warps x one 32 x 32 f32 box
   static constexpr int STG_BYTES = 32 * 32 * 4;
   static constexpr int BARS = STG + 4 * STG_BYTES;
-  // full_I, empty_I, fullT[2], emptyT[2], fullS[2], emptyS[2], s_full, s_empty,
-  // g_full, g_empty, p_full[2], p_empty[2], dxi_full, dxi_empty, drain x 2,
-  // t_full, t_empty
-  static constexpr int NBAR = 24;
+  // full_I, empty_I, slot_full[NSLOT], slot_empty[NSLOT], s_full, s_empty,
+  // g_full[NG], g_empty[NG], p_full[2], p_empty[2], dxi_full, dxi_empty,
+  // drain x 2, t_full, t_empty
+  static constexpr int B_SLOT_FULL = 2, B_SLOT_EMPTY = 2 + NSLOT, B_S = 2 + 2 * NSLOT;
+  static constexpr int B_G_FULL = B_S + 2, B_G_EMPTY = B_G_FULL + NG, B_P = B_G_EMPTY + NG;
+  static constexpr int B_REST = B_P + 4;
+  static constexpr int NBAR = B_REST + 6;
   static constexpr int MISC = BARS + NBAR * 8;
   static constexpr int BYTES = MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
 };
-static_assert(BwdPairSmem::ALLOC <= 232448, "backward shared memory exceeds 227 KB");
+static_assert(BwdPairSmem<false>::ALLOC <= 232448 && BwdPairSmem<true>::ALLOC <= 232448,
+              "backward shared memory exceeds 227 KB");
 // warps 0-15 row, 16-19 epilogue, 20 TMA, 21 logit MMAs, 22 gradient MMAs
 constexpr int BWDP_THREADS = 736;
 // smallest row-block count (N > 4096) that takes the pair kernel
@@ -1181,7 +1196,7 @@ __host__ __device__ __forceinline__ int pair_seq_block(const Unit& U, int m, int
 template <bool SYM>
 __global__ void __launch_bounds__(BWDP_THREADS, 1)
 relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
-  using L = BwdPairSmem;
+  using L = BwdPairSmem<SYM>;
   constexpr int D = 128;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -1194,17 +1209,23 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
   const uint32_t bar0 = base + L::BARS;
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
   const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1);
-  auto FULL_T = [&](int s) { return BAR(2 + s); };
-  auto EMPTY_T = [&](int s) { return BAR(4 + s); };
-  auto FULL_S = [&](int s) { return BAR(6 + s); };
-  auto EMPTY_S = [&](int s) { return BAR(8 + s); };
-  const uint32_t S_FULL = BAR(10), S_EMPTY = BAR(11), G_FULL = BAR(12), G_EMPTY = BAR(13);
-  auto P_FULL = [&](int b) { return BAR(14 + b); };
-  auto P_EMPTY = [&](int b) { return BAR(16 + b); };
-  const uint32_t DXI_FULL = BAR(18), DXI_EMPTY = BAR(19), DRAIN_L = BAR(20), DRAIN_G = BAR(21);
+  // ring use u (X_t[J] of the n-th column tile: u = 2n, X_s[J]: u = 2n + 1) sits
+  // in slot u % 3 and is that slot's (u / 3)-th fill
+  auto SLOT_FULL = [&](uint32_t u) { return BAR(L::B_SLOT_FULL + static_cast<int>(u % L::NSLOT)); };
+  auto SLOT_EMPTY = [&](uint32_t u) { return BAR(L::B_SLOT_EMPTY + static_cast<int>(u % L::NSLOT)); };
+  auto SLOT_PAR = [&](uint32_t u) { return (u / L::NSLOT) & 1u; };
+  const uint32_t S_FULL = BAR(L::B_S), S_EMPTY = BAR(L::B_S + 1);
+  // tile t's G goes to buffer t % NG, that buffer's (t / NG)-th fill
+  auto G_FULL = [&](uint32_t t) { return BAR(L::B_G_FULL + static_cast<int>(t % L::NG)); };
+  auto G_EMPTY = [&](uint32_t t) { return BAR(L::B_G_EMPTY + static_cast<int>(t % L::NG)); };
+  auto G_PAR = [&](uint32_t t) { return (t / L::NG) & 1u; };
+  auto P_FULL = [&](int b) { return BAR(L::B_P + b); };
+  auto P_EMPTY = [&](int b) { return BAR(L::B_P + 2 + b); };
+  const uint32_t DXI_FULL = BAR(L::B_REST), DXI_EMPTY = BAR(L::B_REST + 1);
+  const uint32_t DRAIN_L = BAR(L::B_REST + 2), DRAIN_G = BAR(L::B_REST + 3);
   // causal mask: T_FULL / T_EMPTY guard Z_t, S_FULL / S_EMPTY Z_s; full mask:
   // S_FULL / S_EMPTY guard both
-  const uint32_t T_FULL = BAR(22), T_EMPTY = BAR(23);
+  const uint32_t T_FULL = BAR(L::B_REST + 4), T_EMPTY = BAR(L::B_REST + 5);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::MISC + 4);
 
@@ -1217,21 +1238,21 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
     mbar_init(FULL_I, 1);
     mbar_init(EMPTY_I, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(FULL_T(s), 1);
-      mbar_init(EMPTY_T(s), 1);
       mbar_init(P_FULL(s), 1);
       mbar_init(P_EMPTY(s), 4);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(FULL_S(s), 1);
-      mbar_init(EMPTY_S(s), 1);
+    for (uint32_t b = 0; b < L::NG; ++b) {
+      mbar_init(G_FULL(b), 16);
+      mbar_init(G_EMPTY(b), 1);
+    }
+    for (uint32_t u = 0; u < L::NSLOT; ++u) {
+      mbar_init(SLOT_FULL(u), 1);
+      mbar_init(SLOT_EMPTY(u), 1);
     }
     mbar_init(S_FULL, 1);
     mbar_init(S_EMPTY, 16);
     mbar_init(T_FULL, 1);
     mbar_init(T_EMPTY, 16);
-    mbar_init(G_FULL, 16);
-    mbar_init(G_EMPTY, 1);
     mbar_init(DXI_FULL, 1);
     mbar_init(DXI_EMPTY, 4);
     mbar_init(DRAIN_L, 1);
@@ -1259,7 +1280,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         tma_prefetch_desc(&p.seg[s].tm_dx);
       }
       uint32_t nseq = 0, nJ = 0;
-      uint32_t armsT[2] = {0, 0}, armsS[2] = {0, 0};
+      uint32_t arms[L::NSLOT] = {};
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
         int u, m;
@@ -1285,30 +1306,27 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
           ++nseq;
           const int nT = n_col_tiles64_s<SYM>(p, U, has1 ? R0 + 1 : R0);
           for (int J = 0; J < nT; ++J) {
-            const int tt = nJ & 1, ts = nJ & 1;
-            if (!(ok = mbar_wait(EMPTY_T(tt), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
-            mbar_arrive_expect_tx(FULL_T(tt), L::TILE_J);
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
-              tma_load_4d(base + L::XT_J + tt * L::TILE_J + b * L::BOX_J, &U.seg->tm_t64, FULL_T(tt),
-                          b * 64, U.tok0 + J * BN64, U.h, U.b);
-            ++armsT[tt];
-            if (!(ok = mbar_wait(EMPTY_S(ts), ((nJ >> 1) & 1) ^ 1, wc, W_TMA_EMPTY_J))) break;
-            mbar_arrive_expect_tx(FULL_S(ts), L::TILE_J);
+            for (int which = 0; which < 2; ++which) {   // X_t[J], then X_s[J]
+              const uint32_t use = 2 * nJ + which;
+              const uint32_t slot = use % L::NSLOT;
+              if (!(ok = mbar_wait(SLOT_EMPTY(use), SLOT_PAR(use) ^ 1, wc, W_TMA_EMPTY_J))) break;
+              mbar_arrive_expect_tx(SLOT_FULL(use), L::TILE_J);
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
-              tma_load_4d(base + L::XS_J + ts * L::TILE_J + b * L::BOX_J, &U.seg->tm_s64, FULL_S(ts),
-                          b * 64, U.tok0 + J * BN64, U.h, U.b);
-            ++armsS[ts];
+              for (int b = 0; b < 2; ++b)
+                tma_load_4d(base + L::RING + slot * L::TILE_J + b * L::BOX_J,
+                            which ? &U.seg->tm_s64 : &U.seg->tm_t64, SLOT_FULL(use), b * 64,
+                            U.tok0 + J * BN64, U.h, U.b);
+              ++arms[slot];
+            }
+            if (!ok) break;
             ++nJ;
           }
         }
       }
       if (nseq) mbar_wait_drain(FULL_I, (nseq - 1) & 1, kDrainNs);
-      for (int s = 0; s < 2; ++s)
-        if (armsT[s]) mbar_wait_drain(FULL_T(s), (armsT[s] - 1) & 1, kDrainNs);
-      for (int s = 0; s < 2; ++s)
-        if (armsS[s]) mbar_wait_drain(FULL_S(s), (armsS[s] - 1) & 1, kDrainNs);
+      for (uint32_t k = 0; k < L::NSLOT; ++k)
+        if (arms[k]) mbar_wait_drain(SLOT_FULL(k), (arms[k] - 1) & 1, kDrainNs);
     }
     __syncwarp();
   } else if (warp == BWDP_LOGIT_WARP || warp == BWDP_GRAD_WARP) {
@@ -1328,12 +1346,11 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
     const uint32_t dXsR_k[2] = {sw128_desc_lo(base + L::XS_R0, 16), sw128_desc_lo(base + L::XS_R1, 16)};
     const uint32_t dXsR_mn[2] = {sw128_desc_lo(base + L::XS_R0, L::BOX_I),
                                  sw128_desc_lo(base + L::XS_R1, L::BOX_I)};
-    const uint32_t dXtJ_k0 = sw128_desc_lo(base + L::XT_J, 16);
-    const uint32_t dXsJ_k0 = sw128_desc_lo(base + L::XS_J, 16);
-    const uint32_t dXsJ_mn0 = sw128_desc_lo(base + L::XS_J, L::BOX_J);
+    const uint32_t dRing_k0 = sw128_desc_lo(base + L::RING, 16);
+    const uint32_t dRing_mn0 = sw128_desc_lo(base + L::RING, L::BOX_J);
     const uint32_t dG_k = sw128_desc_lo(base + L::G, 16);
     const uint32_t dG_mn = sw128_desc_lo(base + L::G, L::G_BYTES);
-    constexpr uint32_t J_STEP = L::TILE_J >> 4;
+    constexpr uint32_t J_STEP = L::TILE_J >> 4, G_STEP = L::G_BYTES >> 4;
     uint32_t nseq = 0, nJ = 0, nt = 0, np = 0;
     bool ok = true, issued = false;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -1349,7 +1366,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
         if (!(ok = mbar_wait_warp(FULL_I, nseq & 1, wc, W_MMA_FULL_I))) break;
         bool first_seq = true;
         for (int J = 0; ok && J < nT; ++J) {
-          const int tt = nJ & 1, ts = nJ & 1;
+          const uint32_t ut = 2 * nJ, us = 2 * nJ + 1;   // ring uses of X_t[J], X_s[J]
           for (int rs = 0; rs < 2; ++rs) {
             if (rs == 0 && J >= nT0) continue;
             if (rs == 1 && !has1) continue;
@@ -1359,11 +1376,12 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
               // Z_t, Z_s of tile (R, J) into the logit buffer; under the causal mask
               // Z_t as soon as the row warps have read the previous Z_t, Z_s once
               // they have read the previous Z_s
-              if (!(ok = mbar_wait_warp(FULL_T(tt), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+              if (!(ok = mbar_wait_warp(SLOT_FULL(ut), SLOT_PAR(ut), wc, W_MMA_FULL_J))) break;
               if (!(ok = mbar_wait_warp(SYM ? S_EMPTY : T_EMPTY, (nt & 1) ^ 1, wc, W_MMA_S_EMPTY)))
                 break;
               tc_fence_after();
-              const uint32_t xtj = dXtJ_k0 + tt * J_STEP, xsj = dXsJ_k0 + ts * J_STEP;
+              const uint32_t xtj = dRing_k0 + (ut % L::NSLOT) * J_STEP;
+              const uint32_t xsj = dRing_k0 + (us % L::NSLOT) * J_STEP;
               // K steps: 32 B within a 128 B row, then the next 64-column box
 #pragma unroll
               for (int k = 0; k < D / 16; ++k)
@@ -1371,9 +1389,9 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
                                  HI_1024, xtj + (k >> 2) * (L::BOX_J >> 4) + (k & 3) * 2, HI_1024,
                                  IDESC_S, k > 0 ? 1u : 0u);
               issued = true;
-              if (last_p) umma_commit_lead(lead, EMPTY_T(tt));
+              if (last_p) umma_commit_lead(lead, SLOT_EMPTY(ut));
               if (!SYM) umma_commit_lead(lead, T_FULL);
-              if (!(ok = mbar_wait_warp(FULL_S(ts), (nJ >> 1) & 1, wc, W_MMA_FULL_J))) break;
+              if (!(ok = mbar_wait_warp(SLOT_FULL(us), SLOT_PAR(us), wc, W_MMA_FULL_J))) break;
               if (!SYM && !(ok = mbar_wait_warp(S_EMPTY, (nt & 1) ^ 1, wc, W_MMA_S_EMPTY))) break;
               tc_fence_after();
 #pragma unroll
@@ -1386,29 +1404,31 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
               // dX_R += G X_s[J] and P^T (+)= X_s[R]^T G for tile (R, J).  G_FULL
               // implies the tile's logits (hence its column tiles) are complete.
               const int pb = np & 1;
-              if (!(ok = mbar_wait_warp(G_FULL, nt & 1, wc, W_MMA_G_FULL))) break;
+              const uint32_t gb = nt % L::NG;
+              if (!(ok = mbar_wait_warp(G_FULL(nt), G_PAR(nt), wc, W_MMA_G_FULL))) break;
               if (first_p && !(ok = mbar_wait_warp(P_EMPTY(pb), ((np >> 1) & 1) ^ 1, wc, W_MMA_P_EMPTY)))
                 break;
               if (first_seq && !(ok = mbar_wait_warp(DXI_EMPTY, (nseq & 1) ^ 1, wc, W_MMA_DXI_EMPTY)))
                 break;
               first_seq = false;
               tc_fence_after();
-              const uint32_t xsj = dXsJ_mn0 + ts * J_STEP;
+              const uint32_t xsj = dRing_mn0 + (us % L::NSLOT) * J_STEP;
+              const uint32_t gk = dG_k + gb * G_STEP, gmn = dG_mn + gb * G_STEP;
               // M = i, N = c, K = j (64); K steps of 32 B (G) and 2 KB (X_s[J])
 #pragma unroll
               for (int k = 0; k < BN64 / 16; ++k)
-                umma_bf16_w_lead(lead, tmem + T_DX0 + rs * 128, dG_k + k * 2, HI_1024, xsj + k * 128,
+                umma_bf16_w_lead(lead, tmem + T_DX0 + rs * 128, gk + k * 2, HI_1024, xsj + k * 128,
                                  HI_1024, IDESC_GX, (J > 0 || k > 0) ? 1u : 0u);
               // M = c, N = j, K = i (128); K steps of 2 KB in both
 #pragma unroll
               for (int k = 0; k < BM / 16; ++k)
                 umma_bf16_w_lead(lead, tmem + T_P + pb * 64, dXsR_mn[rs] + k * 128, HI_1024,
-                                 dG_mn + k * 128, HI_1024, IDESC_PT, (!first_p || k > 0) ? 1u : 0u);
+                                 gmn + k * 128, HI_1024, IDESC_PT, (!first_p || k > 0) ? 1u : 0u);
               issued = true;
-              umma_commit_lead(lead, G_EMPTY);
+              umma_commit_lead(lead, G_EMPTY(nt));
               if (last_p) {
                 umma_commit_lead(lead, P_FULL(pb));
-                umma_commit_lead(lead, EMPTY_S(ts));
+                umma_commit_lead(lead, SLOT_EMPTY(us));
                 ++np;
               }
             }
@@ -1527,7 +1547,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
     const int wg = warp >> 2;      // 16-column slice of each 64-column tile
     const int r = q * 32 + lane;
     const float sl2 = p.sl2;
-    const uint32_t gsm = base + L::G + r * 128;  // row r of G: 128 bytes, chunks 2wg, 2wg+1
+    const uint32_t gsm0 = base + L::G + r * 128;  // row r of G: 128 bytes, chunks 2wg, 2wg+1
     uint32_t nt = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
@@ -1615,9 +1635,11 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
               PartnerTile pt{1.f, 1.f, false};
               if (off) pt = partner_tile(pc, btr, bsr);
               form_g_pack<16>(t, s, btr, bsr, mr, col0, limr, off, pc, pt, 0, p, pk);
-              ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
+              // the gradient MMAs of NG tiles back have read this G buffer
+              ok = mbar_wait(G_EMPTY(nt), G_PAR(nt) ^ 1, wc, W_SM_G_EMPTY);
               ok = __all_sync(0xffffffffu, ok);
               if (!ok) break;
+              const uint32_t gsm = gsm0 + (nt % L::NG) * L::G_BYTES;
 #pragma unroll
               for (int h2 = 0; h2 < 2; ++h2) {
                 const int cc = 2 * wg + h2;  // 16-byte chunk within the 128-byte row
@@ -1637,10 +1659,11 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
               }
               pk[k >> 1] = pack_bf16x2(g.x, g.y);
             }
-            // the previous tile's gradient MMAs have read G
-            ok = mbar_wait(G_EMPTY, (nt & 1) ^ 1, wc, W_SM_G_EMPTY);
+            // the gradient MMAs of NG tiles back have read this G buffer
+            ok = mbar_wait(G_EMPTY(nt), G_PAR(nt) ^ 1, wc, W_SM_G_EMPTY);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
+            const uint32_t gsm = gsm0 + (nt % L::NG) * L::G_BYTES;
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int cc = 2 * wg + h2;  // 16-byte chunk within the 128-byte row
@@ -1650,7 +1673,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(G_FULL);
+            if (lane == 0) mbar_arrive(G_FULL(nt));
             ++nt;
           }
         }
@@ -2303,10 +2326,10 @@ cudaError_t tc_launch_bwd(const TcParams& p, int d, int max_grid, cudaStream_t s
   if (q.n_items == 0) return cudaSuccess;
   grid = q.n_items < max_grid ? q.n_items : max_grid;
   auto k = p.causal ? relkl_bwd_pair_kernel<false> : relkl_bwd_pair_kernel<true>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       BwdPairSmem::ALLOC);
+  const int alloc = p.causal ? BwdPairSmem<false>::ALLOC : BwdPairSmem<true>::ALLOC;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
   if (e != cudaSuccess) return e;
-  k<<<grid, BWDP_THREADS, BwdPairSmem::ALLOC, stream>>>(q);
+  k<<<grid, BWDP_THREADS, alloc, stream>>>(q);
   return cudaGetLastError();
 }
 
