@@ -398,7 +398,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="ext_h32_n32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="pipelined end-to-end steps (default: --steps, at least 4; 0 skips)")
     ap.add_argument("--ref-prefix", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
@@ -553,6 +554,10 @@ def main():
     # batch's upload and the last batch's download with the current step; the
     # context-parallel split, whose step holds collectives, runs them in order.
     e2e_ms = None
+    if args.e2e_steps is None:
+        # as many steps as the device timing, so the pipeline's first upload and
+        # last download weigh on the per-step figure no more than K steps allow
+        args.e2e_steps = max(4, args.steps)
     h2d = sum(host[r][0].numel() * host[r][0].element_size() * 2 for r in rels)
     d2h = sum(d.numel() * 4 for d in dx_out) + sum(k.numel() * 4 for k in kl_out)
     if args.e2e_steps > 0 and split != "rows":
