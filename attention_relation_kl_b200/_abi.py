@@ -21,7 +21,7 @@ EXPORTS = ("relkl_workspace_bytes", "relkl_workspace_init", "relkl_fwd", "relkl_
            "relkl_fwd_qkv", "relkl_bwd_qkv", "relkl_get_device_error",
            "relkl_set_wait_timeout_ns", "relkl_status_string", "relkl_last_cuda_error",
            "relkl_path_for", "relkl_fwd_noalloc", "relkl_rope_bwd", "relkl_weight_grad",
-           "relkl_cast_bf16",
+           "relkl_cast_bf16", "relkl_bwd_kernel_for",
            "relkl_fwd_qkv_part", "relkl_bwd_qkv_part", "relkl_check_schedule")
 
 
@@ -86,6 +86,8 @@ def _declare(lib):
     lib.relkl_fwd_noalloc.restype = ctypes.c_int
     lib.relkl_fwd_noalloc.argtypes = [ctypes.POINTER(relkl_desc), _vp, _vp, _vp, _vp, _vp]
     i32 = ctypes.c_int32
+    lib.relkl_bwd_kernel_for.restype = ctypes.c_int32
+    lib.relkl_bwd_kernel_for.argtypes = [ctypes.c_int32, ctypes.POINTER(relkl_desc), ctypes.c_int32]
     lib.relkl_cast_bf16.restype = ctypes.c_int
     lib.relkl_cast_bf16.argtypes = [_vp, _vp, ctypes.c_int64, _vp]
     lib.relkl_rope_bwd.restype = ctypes.c_int

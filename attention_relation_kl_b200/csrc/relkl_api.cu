@@ -27,6 +27,7 @@ cudaError_t launch_cast_bf16(const float* src, void* dst, int64_t n, int num_sms
                              cudaStream_t stream);
 int schedule_check(const TcParams& p0, int d, bool bwd, int n_parts, const int* const* lens,
                    const int* const* offs, char* why, size_t why_len);
+int tc_bwd_kind(const TcParams& p, int d, int sms);
 cudaError_t launch_rope_bwd(const float* dx, void* out, int B, int H, int N, int d, bool bf16_out,
                             double base, double pos_scale, double pos_offset, int apply,
                             cudaStream_t stream);
@@ -607,6 +608,21 @@ relkl_status relkl_check_schedule(int32_t n_rel, const relkl_desc* descs, int32_
   return schedule_check(p, descs[0].d, is_bwd != 0, n_parts, lens, offs, why, why_len) == 0
              ? RELKL_OK
              : RELKL_ERR_INVALID;
+}
+
+int32_t relkl_bwd_kernel_for(int32_t n_rel, const relkl_desc* descs, int32_t n_sms) {
+  if (n_rel < 1 || n_rel > kMaxSeg || !descs || n_sms < 1) return 0;
+  for (int r = 0; r < n_rel; ++r) {
+    if (check_desc(&descs[r]) != RELKL_OK) return 0;
+    if (descs[r].N != descs[0].N || descs[r].causal != descs[0].causal ||
+        (descs[r].cu_seqlens == nullptr) != (descs[0].cu_seqlens == nullptr) ||
+        descs[r].max_seqlen != descs[0].max_seqlen || descs[r].d != descs[0].d)
+      return 0;
+  }
+  if (!tc_shape(descs[0])) return 1;
+  TcParams p;
+  fill_schedule(n_rel, descs, &p, 0, 1);
+  return tc_bwd_kind(p, descs[0].d, n_sms);
 }
 
 relkl_status relkl_rope_bwd(int32_t B, int32_t H, int32_t N, int32_t d, const float* dx_post,

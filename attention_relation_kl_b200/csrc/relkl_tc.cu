@@ -1140,7 +1140,7 @@ relkl_bwd_tc64_kernel(const __grid_constant__ TcParams p) {
 // A work item is the pair sequence k = npb-1-m followed by k = m (npb row-block
 // pairs per unit), which evens out the causal triangle across items.  With
 // few row blocks the items are too coarse to balance 148 SMs, so sequences of
-// at most 32 row blocks use relkl_bwd_tc64_kernel instead.
+// at most 32 row blocks may use relkl_bwd_tc64_kernel instead (tc_bwd_kind).
 template <bool SYM>
 struct BwdPairSmem {
   static constexpr int TILE_I = BM * 128 * 2;        // 128 rows: boxes of 128 x 64 (16 KB)
@@ -1180,8 +1180,10 @@ static_assert(BwdPairSmem<false>::ALLOC <= 232448 && BwdPairSmem<true>::ALLOC <=
               "backward shared memory exceeds 227 KB");
 // warps 0-15 row, 16-19 epilogue, 20 TMA, 21 logit MMAs, 22 gradient MMAs
 constexpr int BWDP_THREADS = 736;
-// smallest row-block count (N > 4096) that takes the pair kernel
-constexpr int kPairMinBlocks = 33;
+// Causal masks at d = 128: sequences of more than 32 row blocks always take the
+// paired-block kernel, sequences of fewer than 16 the one-block kernel, and in
+// between the launch estimates both (tc_bwd_kind).
+constexpr int kPairAlwaysBlocks = 33, kPairMinBlocks = 16;
 constexpr int BWDP_LOGIT_WARP = 21, BWDP_GRAD_WARP = 22;
 
 // Sequence `which` (0 or 1) of pair item m: its first row block, or -1.
@@ -2186,19 +2188,16 @@ struct HostUnitSrc {
 };
 }  // namespace
 
-int schedule_check(const TcParams& p0, int d, bool bwd, int n_parts, const int* const* lens,
-                   const int* const* offs, char* why, size_t why_len) {
+enum SchedKind { FWD, TC64, PAIR, PAIR64 };
+
+static int schedule_check_kind(const TcParams& p0, SchedKind kind, int n_parts,
+                               const int* const* lens, const int* const* offs, char* why,
+                               size_t why_len) {
   const HostUnitSrc src{lens, offs};
   auto fail = [&](const char* what, int u, int R, int J) {
     if (why && why_len) snprintf(why, why_len, "%s (unit %d, row block %d, column tile %d)", what, u, R, J);
     return 1;
   };
-  // which kernel, column tile width, and whether full masks use the symmetric schedule
-  enum { FWD, TC64, PAIR, PAIR64 } kind;
-  if (!bwd) kind = FWD;
-  else if (d == 64) kind = PAIR64;
-  else if (p0.causal && p0.nblk <= kPairMinBlocks - 1) kind = TC64;
-  else kind = PAIR;
   const int W = (kind == FWD || kind == PAIR64) ? 128 : 64;
   const bool tri = p0.causal || (kind == PAIR || kind == PAIR64);   // lower triangle only
   std::vector<std::vector<unsigned char>> seen(p0.n_units);
@@ -2272,6 +2271,54 @@ int schedule_check(const TcParams& p0, int d, bool bwd, int n_parts, const int* 
   return 0;
 }
 
+int schedule_check(const TcParams& p0, int d, bool bwd, int n_parts, const int* const* lens,
+                   const int* const* offs, char* why, size_t why_len) {
+  // the kernels a launch of these shapes may run (the choice between the two
+  // causal d = 128 backwards also depends on the SM count: both are checked)
+  SchedKind kinds[2];
+  int n = 0;
+  if (!bwd) kinds[n++] = FWD;
+  else if (d == 64) kinds[n++] = PAIR64;
+  else if (!p0.causal || p0.nblk >= kPairAlwaysBlocks) kinds[n++] = PAIR;
+  else if (p0.nblk < kPairMinBlocks) kinds[n++] = TC64;
+  else {
+    kinds[n++] = TC64;
+    kinds[n++] = PAIR;
+  }
+  for (int i = 0; i < n; ++i)
+    if (schedule_check_kind(p0, kinds[i], n_parts, lens, offs, why, why_len)) return 1;
+  return 0;
+}
+
+// The paired-block kernels' work items for the part p describes: ceil(npb / 2)
+// per unit, npb = ceil(nblk / 2), shared out like the one-block items.
+static TcParams pair_schedule(const TcParams& p) {
+  TcParams q = p;
+  q.n_pairs = ((p.nblk + 1) / 2 + 1) / 2;
+  q.n_local = q.part < q.n_pairs ? (q.n_pairs - q.part + q.n_parts - 1) / q.n_parts : 0;
+  q.n_items = q.n_units * q.n_local;
+  return q;
+}
+
+// Backward kernel of a tensor-core launch on `sms` SMs: 2 = one 128-row block
+// per pass (relkl_bwd_tc64_kernel), 3 = adjacent row-block pairs
+// (relkl_bwd_pair_kernel), 4 = pairs at d = 64 (relkl_bwd_pair64_kernel).
+// Between 16 and 32 row blocks of a causal mask it compares estimated times:
+// rounds of work items over the SMs times the item's length.  A paired item
+// covers twice the tiles of a one-block item and runs them ~6 % faster
+// (measured at 2K and 4K), so it costs 1.88 one-block items; the one-block
+// kernel's finer items win where the paired kernel's last round would leave
+// many SMs idle (few units: 96 units at N = 4096 run in 11 one-block rounds
+// against 6 paired ones).
+int tc_bwd_kind(const TcParams& p, int d, int sms) {
+  if (d == 64) return 4;
+  if (!p.causal || p.nblk >= kPairAlwaysBlocks) return 3;
+  if (p.nblk < kPairMinBlocks || sms < 1) return 2;
+  const long long one = p.n_items, pair = pair_schedule(p).n_items;
+  const long long r1 = (one + sms - 1) / sms, r2 = (pair + sms - 1) / sms;
+  return r2 * 188 < r1 * 100 ? 3 : 2;
+}
+
 // ------------------------------------------------------------ launchers
 template <int D>
 static cudaError_t launch_fwd(const TcParams& p, int grid, cudaStream_t stream) {
@@ -2291,12 +2338,9 @@ cudaError_t tc_launch_fwd(const TcParams& p, int d, int grid, cudaStream_t strea
 // item of the kernel chosen, whichever is fewer.
 cudaError_t tc_launch_bwd(const TcParams& p, int d, int max_grid, cudaStream_t stream) {
   int grid = p.n_items < max_grid ? p.n_items : max_grid;
-  if (d == 64) {
-    // work items of the paired-block kernel: ceil(npb / 2) per unit
-    TcParams q = p;
-    q.n_pairs = ((p.nblk + 1) / 2 + 1) / 2;
-    q.n_local = q.part < q.n_pairs ? (q.n_pairs - q.part + q.n_parts - 1) / q.n_parts : 0;
-    q.n_items = q.n_units * q.n_local;
+  const int kind = tc_bwd_kind(p, d, max_grid);
+  if (kind == 4) {
+    const TcParams q = pair_schedule(p);
     if (q.n_items == 0) return cudaSuccess;
     grid = q.n_items < max_grid ? q.n_items : max_grid;
     auto k = p.causal ? relkl_bwd_pair64_kernel<false> : relkl_bwd_pair64_kernel<true>;
@@ -2308,8 +2352,8 @@ cudaError_t tc_launch_bwd(const TcParams& p, int d, int max_grid, cudaStream_t s
   }
   // full masks take the paired-block kernel at every N (it serves both
   // orientations of each off-diagonal tile); causal ones with few row blocks
-  // the one-block kernel, whose finer work items balance better
-  if (p.causal && p.nblk <= kPairMinBlocks - 1) {
+  // may take the one-block kernel, whose finer work items balance better
+  if (kind == 2) {
     if (!grid) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(relkl_bwd_tc64_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -2318,11 +2362,7 @@ cudaError_t tc_launch_bwd(const TcParams& p, int d, int max_grid, cudaStream_t s
     relkl_bwd_tc64_kernel<<<grid, BWD_THREADS, Bwd64Smem::ALLOC, stream>>>(p);
     return cudaGetLastError();
   }
-  // work items of the pair kernel: ceil(npb / 2) per unit, npb = ceil(nblk / 2)
-  TcParams q = p;
-  q.n_pairs = ((p.nblk + 1) / 2 + 1) / 2;
-  q.n_local = q.part < q.n_pairs ? (q.n_pairs - q.part + q.n_parts - 1) / q.n_parts : 0;
-  q.n_items = q.n_units * q.n_local;
+  const TcParams q = pair_schedule(p);
   if (q.n_items == 0) return cudaSuccess;
   grid = q.n_items < max_grid ? q.n_items : max_grid;
   auto k = p.causal ? relkl_bwd_pair_kernel<false> : relkl_bwd_pair_kernel<true>;

@@ -58,17 +58,25 @@ def load_peaks():
 FP32_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def bwd_kernel_name(w) -> str:
-    """The backward kernel the library launches for this workload."""
-    if w.dtype != "bf16" or w.d not in (64, 128):
-        return "relkl_bwd_simt_kernel"
-    if w.d == 64:
-        return "relkl_bwd_pair64_kernel"
-    # full masks, and causal ones with more than 32 row blocks, take the kernel
-    # that pairs adjacent row blocks
-    if not w.causal or (w.N + 127) // 128 > 32:
-        return "relkl_bwd_pair_kernel"
-    return "relkl_bwd_tc64_kernel"
+def bwd_kernel_name(w, n_sms: int = 0) -> str:
+    """The backward kernel the library launches for this workload (its own
+    choice, relkl_bwd_kernel_for, on this GPU's SM count; 148 without a GPU)."""
+    from attention_relation_kl_b200 import _abi
+    if n_sms <= 0:
+        n_sms = torch.cuda.get_device_properties(0).multi_processor_count \
+            if torch.cuda.is_available() else 148
+    rels = list(w.relations)
+    descs = (_abi.relkl_desc * len(rels))()
+    for i, r in enumerate(rels):
+        x = descs[i]
+        H = w.heads(r)
+        x.B, x.H, x.N, x.d = w.B, H, w.N, w.d
+        x.stride[0], x.stride[1], x.stride[2], x.stride[3] = H * w.N * w.d, w.N * w.d, w.d, 1
+        x.dtype = _abi.RELKL_BF16 if w.dtype == "bf16" else _abi.RELKL_FP32
+        x.causal, x.scale, x.reserved = 1 if w.causal else 0, 0.0, 0
+    kind = _abi.lib().relkl_bwd_kernel_for(len(rels), descs, n_sms)
+    return {1: "relkl_bwd_simt_kernel", 2: "relkl_bwd_tc64_kernel", 3: "relkl_bwd_pair_kernel",
+            4: "relkl_bwd_pair64_kernel"}[kind]
 
 
 def traffic_record(kernel: str):

@@ -218,6 +218,15 @@ int32_t relkl_last_cuda_error(void);
  * 2 = CUDA-core float32 path, 0 = unsupported.  Validation-free.            */
 int32_t relkl_path_for(const relkl_desc* desc);
 
+/* Which backward kernel relkl_bwd_qkv would launch for these relations on a
+ * GPU with n_sms SMs: 1 = CUDA-core float32 kernel, 2 = one 128-row block per
+ * pass (tensor cores), 3 = adjacent row-block pairs (tensor cores, d = 128),
+ * 4 = adjacent row-block pairs at d = 64; 0 for invalid descs or n_sms < 1.
+ * A causal mask of 16 to 32 row blocks takes 2 or 3 by an estimate of their
+ * times on n_sms SMs; fewer row blocks take 2, more take 3, a full mask 3.
+ * Host only (no device access); validation as in relkl_check_schedule.     */
+int32_t relkl_bwd_kernel_for(int32_t n_rel, const relkl_desc* descs, int32_t n_sms);
+
 /* Forward that needs no workspace from the caller and allocates nothing.
  * The paper has no counterpart: this entry point exists for callers that
  * cannot obtain device memory for a workspace, such as a host framework that

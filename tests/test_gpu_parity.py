@@ -366,6 +366,17 @@ def test_config_full_h32_n16k():
     _sampled(w, units, dx_units=set(units))
 
 
+@pytest.mark.parametrize("N", [2048, 4096])
+def test_config_sweep_short_sequences(N):
+    # the sweep's short-sequence points (B*N = 65536): enough units that the
+    # launch picks the paired-block backward at 16 and 32 row blocks
+    import bench
+    w = workload.sweep_config(N)
+    assert bench.bwd_kernel_name(w) == "relkl_bwd_pair_kernel"
+    units = [("q", 0, 0), ("k", w.B // 2, 17), ("v", w.B - 1, 31)]
+    _sampled(w, units, dx_units=set(units))
+
+
 def test_config_sweep_n64k():
     # the largest point of the sequence-length sweep: B=1, H=32, N=65536
     w = workload.sweep_config(65536)

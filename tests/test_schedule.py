@@ -53,7 +53,7 @@ def _check(descs, is_bwd, n_parts, lens=None, cus=None):
 
 @pytest.mark.parametrize("d,causal,is_bwd", list(itertools.product((64, 128), (True, False), (0, 1))))
 def test_every_tile_once_for_batched_shapes(d, causal, is_bwd):
-    for N in (1, 2, 127, 128, 129, 300, 4096, 4097, 4480, 8197):
+    for N in (1, 2, 127, 128, 129, 300, 2049, 4096, 4097, 4480, 8197):
         for n_parts in (1, 2, 3, 7):
             code, why = _check([_desc(2, 3, N, d, causal)], is_bwd, n_parts)
             assert code == 0, (N, n_parts, why)
@@ -97,3 +97,37 @@ def test_check_refuses_what_it_cannot_replay():
     assert _check([desc], 0, 1)[0] == _abi.RELKL_ERR_INVALID
     assert _check([_desc(1, 1, 100, 96)], 0, 1)[0] == _abi.RELKL_ERR_UNSUPPORTED
     assert _check([_desc(1, 1, 100, 128)], 0, 0)[0] == _abi.RELKL_ERR_INVALID
+
+
+def test_backward_kernel_choice_follows_its_cost_rule():
+    # relkl_bwd_kernel_for against the rule include/relkl.h states: causal d = 128
+    # with 16..32 row blocks takes the paired-block kernel (3) when its rounds of
+    # work items, each 1.88 one-block items long, take less than the one-block
+    # kernel's (2); fewer row blocks take 2, more take 3
+    lib = _abi.lib()
+
+    def choice(descs, sms):
+        return lib.relkl_bwd_kernel_for(len(descs), (relkl_desc * len(descs))(*descs), sms)
+
+    for N in (128, 1920, 2048, 2049, 3000, 4096, 4097, 32768):
+        nblk = (N + 127) // 128
+        for B, H in ((1, 1), (1, 32), (4, 32), (16, 32), (32, 32)):
+            for sms in (148, 132, 8):
+                one = B * H * ((nblk + 1) // 2)
+                pair = B * H * (((nblk + 1) // 2 + 1) // 2)
+                if nblk >= 33:
+                    want = 3
+                elif nblk < 16:
+                    want = 2
+                else:
+                    r1, r2 = -(-one // sms), -(-pair // sms)
+                    want = 3 if r2 * 188 < r1 * 100 else 2
+                assert choice([_desc(B, H, N)], sms) == want, (N, B, H, sms)
+    # the LLaMA2-7B 4K block (Q, K, V of 32 heads: 96 units) keeps the one-block kernel,
+    # the sweep's 16 batches of it take the paired one
+    qkv = [_desc(1, 32, 4096)] * 3
+    assert choice(qkv, 148) == 2 and choice([_desc(16, 32, 4096)] * 3, 148) == 3
+    assert choice([_desc(1, 1, 300, causal=False)], 148) == 3       # full mask
+    assert choice([_desc(1, 1, 300, d=64)], 148) == 4
+    assert choice([_desc(1, 1, 300, d=96)], 148) == 1                # CUDA-core path
+    assert choice([_desc(1, 1, 300)], 0) == 0

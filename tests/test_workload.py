@@ -71,22 +71,15 @@ def test_chain_workload_shapes_determinism_and_projection():
 
 
 def test_bench_names_the_backward_kernel_the_library_launches():
-    # bench.py names the roofline kernel from N; the library picks it with kPairMinBlocks
+    # bench.py asks the library (relkl_bwd_kernel_for) which backward a workload runs
     import os
-    import re
     import sys
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    src = open(os.path.join(root, "attention_relation_kl_b200", "csrc", "relkl_tc.cu")).read()
-    min_blocks = int(re.search(r"constexpr int kPairMinBlocks = (\d+);", src).group(1))
-    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     import bench
-    for N in (128 * (min_blocks - 1), 128 * (min_blocks - 1) + 1, 32768):
-        w = workload.tiny_custom(N=N, d=128, dtype="bf16")
-        want = "relkl_bwd_pair_kernel" if (N + 127) // 128 >= min_blocks else "relkl_bwd_tc64_kernel"
-        assert bench.bwd_kernel_name(w) == want, N
-    # full masks take the paired-block kernel at every N (the symmetric schedule)
-    assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=128, dtype="bf16", causal=False)) \
-        == "relkl_bwd_pair_kernel"
-    assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=64, dtype="bf16")) == \
-        "relkl_bwd_pair64_kernel"
-    assert bench.bwd_kernel_name(workload.tiny_custom(N=300, d=64, dtype="fp32")) == "relkl_bwd_simt_kernel"
+    want = {"ext_h32_n32k": "relkl_bwd_pair_kernel", "gqa_llama3_n16k": "relkl_bwd_pair_kernel",
+            "llama2_h32_n4k": "relkl_bwd_tc64_kernel",      # 96 units: 11 one-block rounds, 6 paired
+            "sweep_n4096": "relkl_bwd_pair_kernel", "sweep_n2048": "relkl_bwd_pair_kernel",
+            "sweep_n1024": "relkl_bwd_tc64_kernel", "full_h32_n16k": "relkl_bwd_pair_kernel",
+            "d64_h32_n32k": "relkl_bwd_pair64_kernel", "tiny_fp32_n256": "relkl_bwd_simt_kernel"}
+    for name, kernel in want.items():
+        assert bench.bwd_kernel_name(workload.get_config(name), n_sms=148) == kernel, name
