@@ -182,7 +182,8 @@ relkl_status relkl_bwd_qkv_part(int32_t n_rel, const relkl_desc* descs,
 
 /* Debug aid, host only (no GPU needed): replays the work decomposition of the
  * tensor-core kernels that a call with these descs would launch (the forward
- * when is_bwd is 0, else the backward the library picks), for every part of
+ * when is_bwd is 0, else the backward the library picks; where that choice
+ * depends on the SM count, see relkl_bwd_kernel_for, both candidates), for every part of
  * n_parts (n_parts = 1: the whole call), and checks that every (unit, row
  * block, column tile) the mask requires is visited exactly once over the
  * parts, that no other tile is, and that every visited tile's TMA row
