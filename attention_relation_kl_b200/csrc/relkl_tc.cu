@@ -1212,7 +1212,7 @@ relkl_bwd_pair_kernel(const __grid_constant__ TcParams p) {
   auto BAR = [&](int i) -> uint32_t { return bar0 + 8u * i; };
   const uint32_t FULL_I = BAR(0), EMPTY_I = BAR(1);
   // ring use u (X_t[J] of the n-th column tile: u = 2n, X_s[J]: u = 2n + 1) sits
-  // in slot u % 3 and is that slot's (u / 3)-th fill
+  // in slot u % NSLOT and is that slot's (u / NSLOT)-th fill
   auto SLOT_FULL = [&](uint32_t u) { return BAR(L::B_SLOT_FULL + static_cast<int>(u % L::NSLOT)); };
   auto SLOT_EMPTY = [&](uint32_t u) { return BAR(L::B_SLOT_EMPTY + static_cast<int>(u % L::NSLOT)); };
   auto SLOT_PAR = [&](uint32_t u) { return (u / L::NSLOT) & 1u; };
