@@ -51,6 +51,20 @@ int main(void) {
   CHECK(relkl_weight_grad(0, 64, 64, f, f, f, f, 256, NULL) == RELKL_ERR_INVALID,
         "weight_grad rows=0");
 
+  /* the bf16 copy of dX_s: n = 0 is a no-op, overlapping ranges are refused */
+  CHECK(relkl_cast_bf16(NULL, NULL, 0, NULL) == RELKL_OK, "cast of nothing");
+  CHECK(relkl_cast_bf16(f, f, 16, NULL) == RELKL_ERR_INVALID, "cast onto its own source");
+  CHECK(relkl_cast_bf16(f, f, -1, NULL) == RELKL_ERR_INVALID, "cast with n < 0");
+
+  /* the backward kernel a launch would pick (host only) */
+  relkl_desc big = desc(1, 32, 32768, 128, RELKL_BF16);
+  relkl_desc d64 = desc(1, 2, 256, 64, RELKL_BF16);
+  CHECK(relkl_bwd_kernel_for(1, &big, 148) == 3, "paired backward at 32K");
+  CHECK(relkl_bwd_kernel_for(1, &tc, 148) == 2, "one-block backward at 2 row blocks");
+  CHECK(relkl_bwd_kernel_for(1, &d64, 148) == 4, "paired d=64 backward");
+  CHECK(relkl_bwd_kernel_for(1, &simt, 148) == 1, "CUDA-core backward");
+  CHECK(relkl_bwd_kernel_for(1, &tc, 0) == 0, "no SMs");
+
   uint64_t old = relkl_set_wait_timeout_ns(123456789ull);
   CHECK(relkl_set_wait_timeout_ns(old) == 123456789ull, "timeout round trip");
   printf("ok %d\n", n_ok);
