@@ -83,3 +83,21 @@ def test_bench_names_the_backward_kernel_the_library_launches():
             "d64_h32_n32k": "relkl_bwd_pair64_kernel", "tiny_fp32_n256": "relkl_bwd_simt_kernel"}
     for name, kernel in want.items():
         assert bench.bwd_kernel_name(workload.get_config(name), n_sms=148) == kernel, name
+
+
+def test_bench_reference_arm_prints_its_line_on_the_host():
+    # bench.py --impl reference times the float64 oracle on the host cores (no GPU)
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "0", "--ref-prefix", "128"],
+                         capture_output=True, text=True, cwd=root, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["config"]["workload"] == "ext_h32_n32k" and line["dtype"] == "f64"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
